@@ -1,0 +1,181 @@
+/*
+ * muon.h - C ABI of the B200 (sm_100a) Muon optimizer step.
+ *
+ * The Muon step for one 2-D hidden-layer weight W (rows x cols) with gradient g:
+ *
+ *   g <- g - 1 mean_dim0(g)^T                  optional zero-centring, before momentum
+ *                                              ("Muon meets Mamba", sections 2.1 and 4.2)
+ *   m <- mu m + (1 - mu) g                     momentum buffer (EMA form)
+ *   u <- nesterov ? mu m + (1 - mu) g : m      Nesterov look-ahead
+ *                                              ("Muon optimizer: matrix-aware LLM training",
+ *                                               `Muon.step` listing)
+ *   X <- u / (||u||_F + eps), transposed when rows > cols
+ *   repeat steps times:                        ("Muon optimizer ..." `newtonschulz5` listing;
+ *     A <- X X^T                                "AdamW vs Muon" part 3, the quintic update
+ *     B <- b_k A + c_k A A                      M_k = a M + b (M M^T) M + c (M M^T)^2 M)
+ *     X <- a_k X + B X
+ *   O <- X, transposed back
+ *   W <- W (1 - lr wd) - lr s O               decoupled decay and update; s is the RMS factor
+ *                                              ("AdamW vs Muon" part 3 "scaling and update";
+ *                                               "Muon meets Mamba" section 4.2)
+ *
+ * All arithmetic runs in hand-written sm_100a kernels: a fused elementwise prologue, the
+ * Newton-Schulz matrix products on the tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation in tensor memory), and a fused elementwise epilogue. There is no CPU fallback:
+ * on a machine without an sm_100 device every compute call fails with MUON_ERR_UNSUPPORTED.
+ *
+ * Conventions shared by every call:
+ *   - Matrices are dense, row-major, contiguous (leading dimension = cols).
+ *   - Pointers named "device" must be device memory (or managed memory) of the current device.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ *     never synchronise the host, except the first call with a new set of shapes, which
+ *     allocates the library's workspace (cudaMalloc) and uploads its tables.
+ *   - The workspace is owned by the library, per process, and shared by all calls: calls must be
+ *     ordered (same stream, or synchronised by the caller). Concurrent calls race.
+ *   - Argument errors are detected before any device work is enqueued; the call then returns a
+ *     negative code and muon_last_error() describes the first problem found.
+ *   - Device-side faults of the library's own making (a wait that timed out inside a kernel, a
+ *     non-finite value in an update matrix) are recorded in a device status word that
+ *     muon_check_status() reads.
+ */
+#ifndef MUON_H_
+#define MUON_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so that this header needs no CUDA headers. */
+typedef struct CUstream_st* muon_stream_t;
+
+typedef enum { MUON_BF16 = 0, MUON_FP32 = 1 } muon_dtype_t;
+
+/* Working precision of the Newton-Schulz iterate.
+ *   MUON_PREC_BF16: X, A, B stored in bf16, products on tcgen05 tensor cores with fp32
+ *                   accumulation (the pages' bf16 working copy).
+ *   MUON_PREC_FP32: X, A, B stored in fp32, products as fp32 FMA on the CUDA cores
+ *                   (a correctness mode; no speed target). */
+typedef enum { MUON_PREC_BF16 = 0, MUON_PREC_FP32 = 1 } muon_prec_t;
+
+/* RMS factor s of the update ("AdamW vs Muon" part 3 rescales by matrix shape without giving a
+ * formula): MUON_RMS_ONE gives s = 1; MUON_RMS_SQRT_MAX1_ROWS_OVER_COLS gives
+ * s = sqrt(max(1, rows / cols)). */
+typedef enum { MUON_RMS_ONE = 0, MUON_RMS_SQRT_MAX1_ROWS_OVER_COLS = 1 } muon_rms_t;
+
+/* One Newton-Schulz iteration's coefficients: X <- a X + b (X X^T) X + c (X X^T)^2 X.
+ * Quintic ("Muon optimizer ..." `newtonschulz5`): {3.4445, -4.7750, 2.0315}.
+ * Cubic ("Muon meets Mamba" 2.2):                 {1.5, -0.5, 0}.
+ * When c == 0 the A A product is skipped. */
+typedef struct {
+  float a, b, c;
+} muon_coeffs_t;
+
+/* Return codes. */
+enum {
+  MUON_OK = 0,
+  MUON_WARN_NONFINITE = 1,    /* muon_check_status only: a NaN/Inf reached an update matrix   */
+  MUON_ERR_INVALID_ARG = -1,  /* bad pointer, size, count, step count or aliasing             */
+  MUON_ERR_UNSUPPORTED = -2,  /* no sm_100 device, or a dtype/precision combination not built  */
+  MUON_ERR_WORKSPACE = -3,    /* workspace allocation failed (device out of memory)           */
+  MUON_ERR_CUDA = -4,         /* a CUDA runtime/driver call failed                            */
+  MUON_ERR_TIMEOUT = -5       /* muon_check_status only: a kernel wait hit its time limit and  */
+                              /* the kernel returned early; results of that call are invalid  */
+};
+
+/* Largest number of Newton-Schulz iterations accepted by one call. */
+#define MUON_MAX_NS_STEPS 64
+
+/*
+ * Newton-Schulz orthogonalisation of one matrix ("Muon optimizer ..." `newtonschulz5`).
+ *
+ *   G      device, m x n (m rows, n cols), element type g_dtype. Read only.
+ *   X      device, m x n, element type x_dtype. Written: X = NS(G). May not overlap G.
+ *   steps  number of iterations, 0..MUON_MAX_NS_STEPS; 0 returns G / (||G||_F + eps).
+ *   coeffs host array of `steps` triples, or NULL for `steps` quintic triples.
+ *   zero_center  nonzero: subtract the mean over dim 0 (column means) from G first.
+ *   eps    added to the Frobenius norm before dividing (pages: 1e-7). Must be >= 0.
+ *   prec   working precision (see muon_prec_t).
+ * Rows > cols runs the iteration on G^T and transposes back, as the pages do.
+ * Returns MUON_OK or a negative error code.
+ */
+MUON_API int muon_ns_orthogonalize(const void* G, muon_dtype_t g_dtype, void* X, muon_dtype_t x_dtype,
+                          int64_t m, int64_t n, int steps, const muon_coeffs_t* coeffs,
+                          int zero_center, float eps, muon_prec_t prec, muon_stream_t stream);
+
+/*
+ * One Muon step over `count` independent matrices ("Muon optimizer ..." `Muon.step`;
+ * "Muon meets Mamba" section 4.2 `_step_muon`).
+ *
+ *   params[i]   device fp32, rows[i] x cols[i]; updated in place.
+ *   grads[i]    device, element type grad_dtype; read only. NULL skips matrix i entirely
+ *               (its params and momentum are left untouched), like a parameter with no grad.
+ *   momentum[i] device fp32, same shape; updated in place. Start from zeros.
+ *               (The pages keep the buffer in the gradient's dtype; fp32 is used here so that
+ *               the parameter update stays accurate.)
+ *   lr, mu, nesterov, weight_decay   as in the step above; 0 <= mu < 1, lr and wd finite.
+ *   rms_scale   the RMS factor s (muon_rms_t).
+ *   steps, coeffs, zero_center, eps, prec   as for muon_ns_orthogonalize.
+ * params[i] and momentum[i] must not overlap each other or any other matrix's buffers.
+ * All `count` matrices are processed by the same kernel launches (one prologue, one grouped
+ * tensor-core launch per Newton-Schulz phase, one epilogue), so small matrices are not
+ * launch-bound. Returns MUON_OK or a negative error code.
+ */
+MUON_API int muon_step(int count, float* const* params, const void* const* grads, muon_dtype_t grad_dtype,
+              float* const* momentum, const int64_t* rows, const int64_t* cols, float lr, float mu,
+              int nesterov, float weight_decay, muon_rms_t rms_scale, int steps,
+              const muon_coeffs_t* coeffs, int zero_center, float eps, muon_prec_t prec,
+              muon_stream_t stream);
+
+/* Message describing the last error returned on the calling thread ("" if none). The pointer
+ * stays valid until the next call on that thread. */
+MUON_API const char* muon_last_error(void);
+
+/* Synchronises `stream`, then reads and clears the device status word of the current device.
+ * Returns MUON_ERR_TIMEOUT if a kernel gave up waiting since the last check,
+ * MUON_WARN_NONFINITE if a NaN or Inf reached an update matrix, MUON_OK otherwise
+ * (or MUON_ERR_CUDA if synchronising failed). */
+MUON_API int muon_check_status(muon_stream_t stream);
+
+/* Frees the workspace and cached plans of the current device (synchronises the device). */
+MUON_API int muon_release_workspace(void);
+
+/* Kernel classes counted and timed by the library, indices into muon_profile_read's arrays. */
+enum {
+  MUON_KC_CENTER = 0,   /* column sums and means for zero-centring                    */
+  MUON_KC_PROLOGUE = 1, /* momentum, Nesterov, norm partials, bf16 cast                 */
+  MUON_KC_NORM = 2,     /* per-matrix 1 / (||u|| + eps)                                 */
+  MUON_KC_GEMM = 3,     /* Newton-Schulz matrix products (all three phases)             */
+  MUON_KC_EPILOGUE = 4, /* decay and parameter update, or the output conversion         */
+  MUON_KC_COUNT = 5
+};
+
+/* Turns per-launch timing on (nonzero) or off. While on, every kernel launch is bracketed by
+ * CUDA events recorded on the launching stream. */
+MUON_API int muon_profile_enable(int on);
+
+/* Synchronises the recorded events and returns, per kernel class, the number of launches and
+ * their summed device time in milliseconds since the last read (arrays of MUON_KC_COUNT).
+ * Also returns, in flops (may be NULL), the nominal Newton-Schulz FLOPs of those GEMM launches
+ * (4 m^2 n + 2 m^3 per quintic iteration, m = min dim) and, in exec_flops (may be NULL), the
+ * FLOPs the tensor cores actually executed (triangle tiles only). Clears the records. */
+MUON_API int muon_profile_read(int64_t* launches, double* ms, double* flops, double* exec_flops);
+
+/* Total number of kernels this library has launched in this process. */
+MUON_API int64_t muon_launch_count(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+MUON_API int muon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_H_ */

@@ -1,0 +1,788 @@
+// C ABI of the Muon step (see include/muon.h): argument validation, the per-device plan
+// (workspace layout, TMA descriptors, grouped problem tables) and the launch sequence.
+//
+// Launch sequence of one muon_step (all on the caller's stream, no host synchronisation once the
+// plan exists):
+//   [column sums, column means]   only with zero-centring
+//   prologue                      momentum, Nesterov, norm partials, U = cast(u)
+//   norm                          alpha_j = 1 / (||u_j||_F + eps)
+//   per Newton-Schulz iteration k (one grouped launch per phase covering every matrix):
+//     gram     A = X X^T                (k = 0: scaled by alpha^2, folding the normalisation)
+//     poly     B = b_k A + c_k A A      (skipped when c_k = 0)
+//     update   X' = a_k X + B X         (k = 0: scaled by alpha; c_k = 0: X' = a_k X + b_k A X)
+//   epilogue                      p = p (1 - lr wd) - lr s O
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/muon.h"
+#include "muon_internal.h"
+
+namespace muon {
+
+size_t gemm_tc_smem_bytes();
+
+namespace {
+
+thread_local std::string t_err;
+std::mutex g_mu;
+int64_t g_launches = 0;
+
+int fail(int code, const std::string& msg) {
+  t_err = msg;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MUON_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+#define MUON_CUDA(expr)                                   \
+  do {                                                    \
+    cudaError_t e_ = (expr);                              \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #expr);   \
+  } while (0)
+
+// ------------------------------------------------------------------ profiling
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, exec;
+};
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t get_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+template <class F>
+cudaError_t timed_launch(int kind, cudaStream_t s, double flops, double exec, F&& launch) {
+  ++g_launches;
+  if (!g_prof_on) return launch();
+  ProfRec r{kind, get_event(), get_event(), flops, exec};
+  cudaEventRecord(r.a, s);
+  cudaError_t e = launch();
+  cudaEventRecord(r.b, s);
+  g_prof.push_back(r);
+  return e;
+}
+
+// ------------------------------------------------------------------ driver entry point
+typedef CUresult (*PFN_encodeTiled_t)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                      const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                      CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled_t get_encode() {
+  static PFN_encodeTiled_t fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled_t>(p);
+  }
+  return fn;
+}
+
+// ------------------------------------------------------------------ plan
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct Shape {
+  int64_t r, c;
+  bool operator==(const Shape& o) const { return r == o.r && c == o.c; }
+};
+
+struct BufMaps {   // three TMA views of one bf16 buffer
+  int k128 = -1, k256 = -1, mn64 = -1;
+};
+
+struct Plan {
+  std::vector<Shape> shapes;
+  int x_bf16 = 1;
+  int dev = -1;
+  char* ws = nullptr;
+  size_t ws_bytes = 0;
+  // device tables
+  MatInfo* d_mats = nullptr;
+  float* d_partials = nullptr;
+  int64_t n_chunks = 0, cs_items = 0, cm_items = 0;
+  // per-matrix workspace pointers
+  std::vector<void*> x0, x1, A, B;
+  std::vector<float*> colmean, colpart, alpha;
+  std::vector<int64_t> ldx, ldm;
+  // grouped problems
+  void* d_gram[2] = {nullptr, nullptr};
+  void* d_poly = nullptr;
+  void* d_updB[2] = {nullptr, nullptr};
+  void* d_updA[2] = {nullptr, nullptr};
+  uint32_t tiles_gram = 0, tiles_poly = 0, tiles_upd = 0;
+  double fl_gram = 0, fl_poly = 0, fl_upd = 0;      // nominal flops per launch
+  double ex_gram = 0, ex_poly = 0, ex_upd = 0;      // executed (tile) flops per launch
+  // per-call MatInfo staging
+  std::vector<MatInfo> last_uploaded;
+  MatInfo* h_pinned = nullptr;
+  cudaEvent_t upload_done = nullptr;
+  bool uploaded_once = false;
+
+  ~Plan() {
+    if (upload_done) cudaEventDestroy(upload_done);
+    if (h_pinned) cudaFreeHost(h_pinned);
+    if (ws) cudaFree(ws);
+  }
+};
+
+struct DeviceState {
+  std::unique_ptr<Plan> plan;
+  int* d_status = nullptr;  // [0] flags, [1] non-finite count
+  int sms = 0;
+  int cc_major = 0;
+};
+
+std::map<int, DeviceState> g_dev;
+
+int device_state(DeviceState** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MUON_ERR_UNSUPPORTED, std::string("no CUDA device: ") + cudaGetErrorString(e));
+  DeviceState& ds = g_dev[dev];
+  if (ds.sms == 0) {
+    cudaDeviceProp prop;
+    MUON_CUDA(cudaGetDeviceProperties(&prop, dev));
+    ds.sms = prop.multiProcessorCount;
+    ds.cc_major = prop.major;
+  }
+  if (ds.cc_major != 10)
+    return fail(MUON_ERR_UNSUPPORTED, "this library runs on sm_100 (B200) devices only");
+  if (!ds.d_status) {
+    MUON_CUDA(cudaMalloc(&ds.d_status, 2 * sizeof(int)));
+    MUON_CUDA(cudaMemset(ds.d_status, 0, 2 * sizeof(int)));
+  }
+  *out = &ds;
+  return MUON_OK;
+}
+
+// Builds the workspace, TMA descriptors and grouped problem tables for a list of shapes.
+int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Plan** out) {
+  int dev = 0;
+  MUON_CUDA(cudaGetDevice(&dev));
+  if (ds.plan && ds.plan->shapes == shapes && ds.plan->x_bf16 == x_bf16) {
+    *out = ds.plan.get();
+    return MUON_OK;
+  }
+  ds.plan.reset();  // frees the previous workspace (cudaFree synchronises)
+  std::unique_ptr<Plan> P(new Plan());
+  P->shapes = shapes;
+  P->x_bf16 = x_bf16;
+  P->dev = dev;
+  const int n = (int)shapes.size();
+  const size_t esz = x_bf16 ? 2 : 4;
+  const size_t AL = 256;
+
+  // ---- layout
+  size_t off = 0;
+  std::vector<size_t> o_x0(n), o_x1(n), o_A(n), o_B(n), o_cm(n), o_cp(n);
+  P->ldx.resize(n);
+  P->ldm.resize(n);
+  int64_t chunks = 0, cs = 0, cm = 0;
+  std::vector<MatInfo> mats(n);
+  for (int j = 0; j < n; ++j) {
+    const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c);
+    const int64_t ldx = align_up(c, 8), ldm = align_up(m, 8);
+    P->ldx[j] = ldx;
+    P->ldm[j] = ldm;
+    o_x0[j] = off; off = align_up(off + (size_t)r * ldx * esz, AL);
+    o_x1[j] = off; off = align_up(off + (size_t)r * ldx * esz, AL);
+    o_A[j] = off; off = align_up(off + (size_t)m * ldm * esz, AL);
+    o_B[j] = off; off = align_up(off + (size_t)m * ldm * esz, AL);
+    o_cm[j] = off; off = align_up(off + (size_t)c * 4, AL);
+    const int64_t n_rc = ceil_div(r, kCsRows), n_cb = ceil_div(c, kCsCols);
+    o_cp[j] = off; off = align_up(off + (size_t)n_rc * c * 4, AL);
+    MatInfo& mi = mats[j];
+    std::memset(&mi, 0, sizeof(mi));
+    mi.rows = r; mi.cols = c; mi.ldx = ldx;
+    mi.chunk_begin = chunks; chunks += ceil_div(r * c, kChunk);
+    mi.cs_begin = cs; cs += n_rc * n_cb;
+    mi.cm_begin = cm; cm += n_cb;
+  }
+  const size_t o_alpha = off; off = align_up(off + (size_t)n * 4, AL);
+  const size_t o_part = off; off = align_up(off + (size_t)chunks * 4, AL);
+  const size_t o_mats = off; off = align_up(off + (size_t)n * sizeof(MatInfo), AL);
+  const int maps_per = 12;
+  const size_t o_maps = off;
+  if (x_bf16) off = align_up(off + (size_t)n * maps_per * sizeof(CUtensorMap), AL);
+  const size_t prob_sz = x_bf16 ? sizeof(GemmProblem) : sizeof(GemmProblemF32);
+  size_t o_prob[7];
+  for (int k = 0; k < 7; ++k) { o_prob[k] = off; off = align_up(off + (size_t)n * prob_sz, AL); }
+  P->ws_bytes = off;
+
+  cudaError_t e = cudaMalloc(&P->ws, P->ws_bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    char buf[160];
+    snprintf(buf, sizeof(buf), "workspace allocation of %.3f GB failed: %s", P->ws_bytes / 1e9,
+             cudaGetErrorString(e));
+    return fail(MUON_ERR_WORKSPACE, buf);
+  }
+  char* W = P->ws;
+  P->n_chunks = chunks;
+  P->cs_items = cs;
+  P->cm_items = cm;
+  P->d_partials = reinterpret_cast<float*>(W + o_part);
+  P->d_mats = reinterpret_cast<MatInfo*>(W + o_mats);
+  for (int j = 0; j < n; ++j) {
+    P->x0.push_back(W + o_x0[j]);
+    P->x1.push_back(W + o_x1[j]);
+    P->A.push_back(W + o_A[j]);
+    P->B.push_back(W + o_B[j]);
+    P->colmean.push_back(reinterpret_cast<float*>(W + o_cm[j]));
+    P->colpart.push_back(reinterpret_cast<float*>(W + o_cp[j]));
+    P->alpha.push_back(reinterpret_cast<float*>(W + o_alpha) + j);
+  }
+
+  // ---- grouped problems
+  auto sym_tiles = [](int64_t m) {
+    const int64_t tm = ceil_div(m, kTcBM), tn = ceil_div(m, kTcBN);
+    int64_t t = 0;
+    for (int64_t bi = 0; bi < tm; ++bi) t += tn - bi / 2;
+    return t;
+  };
+  if (x_bf16) {
+    PFN_encodeTiled_t encode = get_encode();
+    if (!encode) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    std::vector<CUtensorMap> maps((size_t)n * maps_per);
+    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(W + o_maps);
+    int bad = 0;
+    auto make3 = [&](int j, int slot, void* base, int64_t rows, int64_t cols, int64_t ld) {
+      BufMaps bm;
+      const int boxes[3] = {kTcBM, kTcBN, 64};
+      int* dst[3] = {&bm.k128, &bm.k256, &bm.mn64};
+      for (int b = 0; b < 3; ++b) {
+        const int idx = j * maps_per + slot * 3 + b;
+        cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+        cuuint64_t gstride[1] = {(cuuint64_t)(ld * 2)};
+        cuuint32_t box[2] = {64u, (cuuint32_t)boxes[b]};
+        cuuint32_t estr[2] = {1u, 1u};
+        CUresult r = encode(&maps[idx], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, gdim, gstride, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) bad = (int)r;
+        *dst[b] = idx;
+      }
+      return bm;
+    };
+    std::vector<GemmProblem> gram[2], poly, updB[2], updA[2];
+    uint32_t tg = 0, tp = 0, tu = 0;
+    for (int j = 0; j < n; ++j) {
+      const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c), nn = std::max(r, c);
+      const bool tall = r > c;
+      BufMaps mx[2] = {make3(j, 0, P->x0[j], r, c, P->ldx[j]), make3(j, 1, P->x1[j], r, c, P->ldx[j])};
+      BufMaps mA = make3(j, 2, P->A[j], m, m, P->ldm[j]);
+      BufMaps mB = make3(j, 3, P->B[j], m, m, P->ldm[j]);
+      auto M_ = [&](int idx) { return d_maps + idx; };
+      for (int p = 0; p < 2; ++p) {
+        GemmProblem g{};
+        g.tma_a = M_(tall ? mx[p].mn64 : mx[p].k128);
+        g.tma_b = M_(tall ? mx[p].mn64 : mx[p].k256);
+        g.a_mn = g.b_mn = tall ? 1 : 0;
+        g.d = static_cast<__nv_bfloat16*>(P->A[j]);
+        g.ldd = P->ldm[j];
+        g.alpha = P->alpha[j];
+        g.M = g.N = (uint32_t)m;
+        g.K = (uint32_t)nn;
+        g.tiles_m = (uint32_t)ceil_div(m, kTcBM);
+        g.tiles_n = (uint32_t)ceil_div(m, kTcBN);
+        g.sym = 1;
+        g.n_tiles = (uint32_t)sym_tiles(m);
+        g.tile_begin = tg;
+        gram[p].push_back(g);
+        for (int which = 0; which < 2; ++which) {   // 0: operand B, 1: operand A
+          void* S = which == 0 ? P->B[j] : P->A[j];
+          const BufMaps& mS = which == 0 ? mB : mA;
+          (void)S;
+          GemmProblem u{};
+          if (!tall) {
+            u.tma_a = M_(mS.k128); u.a_mn = 0;
+            u.tma_b = M_(mx[p].mn64); u.b_mn = 1;
+          } else {
+            u.tma_a = M_(mx[p].k128); u.a_mn = 0;
+            u.tma_b = M_(mS.k256); u.b_mn = 0;
+          }
+          u.d = static_cast<__nv_bfloat16*>(p == 0 ? P->x1[j] : P->x0[j]);
+          u.ldd = P->ldx[j];
+          u.c = static_cast<const __nv_bfloat16*>(p == 0 ? P->x0[j] : P->x1[j]);
+          u.ldc = P->ldx[j];
+          u.alpha = P->alpha[j];
+          u.M = (uint32_t)r; u.N = (uint32_t)c; u.K = (uint32_t)m;
+          u.tiles_m = (uint32_t)ceil_div(r, kTcBM);
+          u.tiles_n = (uint32_t)ceil_div(c, kTcBN);
+          u.n_tiles = u.tiles_m * u.tiles_n;
+          u.tile_begin = tu;
+          (which == 0 ? updB[p] : updA[p]).push_back(u);
+        }
+      }
+      GemmProblem q{};
+      q.tma_a = M_(mA.k128); q.tma_b = M_(mA.k256);
+      q.d = static_cast<__nv_bfloat16*>(P->B[j]); q.ldd = P->ldm[j];
+      q.c = static_cast<const __nv_bfloat16*>(P->A[j]); q.ldc = P->ldm[j];
+      q.alpha = P->alpha[j];
+      q.M = q.N = q.K = (uint32_t)m;
+      q.tiles_m = (uint32_t)ceil_div(m, kTcBM); q.tiles_n = (uint32_t)ceil_div(m, kTcBN);
+      q.sym = 1;
+      q.n_tiles = (uint32_t)sym_tiles(m);
+      q.tile_begin = tp;
+      poly.push_back(q);
+      tg += gram[0].back().n_tiles;
+      tp += q.n_tiles;
+      tu += updB[0].back().n_tiles;
+      P->fl_gram += 2.0 * m * m * nn;
+      P->fl_poly += 2.0 * m * m * m;
+      P->fl_upd += 2.0 * m * m * nn;
+      const double tile_fl = 2.0 * kTcBM * kTcBN;
+      P->ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kTcBK) * kTcBK);
+      P->ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
+      P->ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
+    }
+    if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
+    P->tiles_gram = tg; P->tiles_poly = tp; P->tiles_upd = tu;
+    MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+    std::vector<GemmProblem>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
+    void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
+                      &P->d_updA[0], &P->d_updA[1]};
+    for (int k = 0; k < 7; ++k) {
+      *dsts[k] = W + o_prob[k];
+      MUON_CUDA(cudaMemcpy(*dsts[k], lists[k]->data(), lists[k]->size() * sizeof(GemmProblem),
+                           cudaMemcpyHostToDevice));
+    }
+  } else {
+    std::vector<GemmProblemF32> gram[2], poly, updB[2], updA[2];
+    uint32_t tg = 0, tp = 0, tu = 0;
+    for (int j = 0; j < n; ++j) {
+      const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c), nn = std::max(r, c);
+      const bool tall = r > c;
+      const int64_t ldx = P->ldx[j], ldm = P->ldm[j];
+      float* X[2] = {static_cast<float*>(P->x0[j]), static_cast<float*>(P->x1[j])};
+      float* A = static_cast<float*>(P->A[j]);
+      float* B = static_cast<float*>(P->B[j]);
+      for (int p = 0; p < 2; ++p) {
+        GemmProblemF32 g{};
+        g.a = g.b = X[p];
+        if (!tall) { g.sa_i = g.sb_j = ldx; g.sa_k = g.sb_k = 1; }
+        else { g.sa_i = g.sb_j = 1; g.sa_k = g.sb_k = ldx; }
+        g.d = A; g.ldd = ldm; g.alpha = P->alpha[j];
+        g.M = g.N = (uint32_t)m; g.K = (uint32_t)nn;
+        g.tiles_m = g.tiles_n = (uint32_t)ceil_div(m, kF32BM);
+        g.n_tiles = g.tiles_m * g.tiles_n;
+        g.tile_begin = tg;
+        gram[p].push_back(g);
+        for (int which = 0; which < 2; ++which) {
+          float* S = which == 0 ? B : A;
+          GemmProblemF32 u{};
+          if (!tall) {
+            u.a = S; u.sa_i = ldm; u.sa_k = 1;
+            u.b = X[p]; u.sb_j = 1; u.sb_k = ldx;
+          } else {
+            u.a = X[p]; u.sa_i = ldx; u.sa_k = 1;
+            u.b = S; u.sb_j = ldm; u.sb_k = 1;
+          }
+          u.d = X[1 - p]; u.ldd = ldx;
+          u.c = X[p]; u.ldc = ldx;
+          u.alpha = P->alpha[j];
+          u.M = (uint32_t)r; u.N = (uint32_t)c; u.K = (uint32_t)m;
+          u.tiles_m = (uint32_t)ceil_div(r, kF32BM); u.tiles_n = (uint32_t)ceil_div(c, kF32BN);
+          u.n_tiles = u.tiles_m * u.tiles_n;
+          u.tile_begin = tu;
+          (which == 0 ? updB[p] : updA[p]).push_back(u);
+        }
+      }
+      GemmProblemF32 q{};
+      q.a = q.b = A; q.sa_i = q.sb_j = ldm; q.sa_k = q.sb_k = 1;
+      q.d = B; q.ldd = ldm; q.c = A; q.ldc = ldm; q.alpha = P->alpha[j];
+      q.M = q.N = q.K = (uint32_t)m;
+      q.tiles_m = q.tiles_n = (uint32_t)ceil_div(m, kF32BM);
+      q.n_tiles = q.tiles_m * q.tiles_n;
+      q.tile_begin = tp;
+      poly.push_back(q);
+      tg += gram[0].back().n_tiles;
+      tp += q.n_tiles;
+      tu += updB[0].back().n_tiles;
+      P->fl_gram += 2.0 * m * m * nn;
+      P->fl_poly += 2.0 * m * m * m;
+      P->fl_upd += 2.0 * m * m * nn;
+    }
+    P->ex_gram = P->fl_gram; P->ex_poly = P->fl_poly; P->ex_upd = P->fl_upd;
+    P->tiles_gram = tg; P->tiles_poly = tp; P->tiles_upd = tu;
+    std::vector<GemmProblemF32>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
+    void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
+                      &P->d_updA[0], &P->d_updA[1]};
+    for (int k = 0; k < 7; ++k) {
+      *dsts[k] = W + o_prob[k];
+      MUON_CUDA(cudaMemcpy(*dsts[k], lists[k]->data(), lists[k]->size() * sizeof(GemmProblemF32),
+                           cudaMemcpyHostToDevice));
+    }
+  }
+
+  // ---- per-call table staging
+  MUON_CUDA(cudaMallocHost(&P->h_pinned, (size_t)n * sizeof(MatInfo)));
+  MUON_CUDA(cudaEventCreateWithFlags(&P->upload_done, cudaEventDisableTiming));
+  for (int j = 0; j < n; ++j) {
+    mats[j].x0 = P->x0[j];
+    mats[j].colmean = P->colmean[j];
+    mats[j].colpart = P->colpart[j];
+    mats[j].alpha = P->alpha[j];
+  }
+  P->last_uploaded = mats;   // template: pointers of the call are filled in per call
+  ds.plan = std::move(P);
+  *out = ds.plan.get();
+  return MUON_OK;
+}
+
+// Fills the per-call fields and uploads the table when it differs from the last upload.
+int upload_mats(Plan& P, std::vector<MatInfo>& mats, cudaStream_t s) {
+  if (P.uploaded_once && std::memcmp(mats.data(), P.last_uploaded.data(), mats.size() * sizeof(MatInfo)) == 0)
+    return MUON_OK;
+  MUON_CUDA(cudaEventSynchronize(P.upload_done));
+  std::memcpy(P.h_pinned, mats.data(), mats.size() * sizeof(MatInfo));
+  MUON_CUDA(cudaMemcpyAsync(P.d_mats, P.h_pinned, mats.size() * sizeof(MatInfo), cudaMemcpyHostToDevice, s));
+  MUON_CUDA(cudaEventRecord(P.upload_done, s));
+  P.last_uploaded = mats;
+  P.uploaded_once = true;
+  return MUON_OK;
+}
+
+bool finite_f(float x) { return std::isfinite(x); }
+
+int check_coeffs(int steps, const muon_coeffs_t* coeffs, std::vector<muon_coeffs_t>& out) {
+  if (steps < 0 || steps > MUON_MAX_NS_STEPS)
+    return fail(MUON_ERR_INVALID_ARG, "steps must be in [0, " + std::to_string(MUON_MAX_NS_STEPS) + "]");
+  out.resize(steps);
+  for (int k = 0; k < steps; ++k) {
+    out[k] = coeffs ? coeffs[k] : muon_coeffs_t{3.4445f, -4.7750f, 2.0315f};
+    if (!finite_f(out[k].a) || !finite_f(out[k].b) || !finite_f(out[k].c))
+      return fail(MUON_ERR_INVALID_ARG, "coefficients must be finite");
+  }
+  return MUON_OK;
+}
+
+int check_shape(int64_t r, int64_t c, const char* what) {
+  if (r <= 0 || c <= 0)
+    return fail(MUON_ERR_INVALID_ARG, std::string(what) + ": rows and cols must be positive");
+  if (r > (1 << 20) || c > (1 << 20) || r * c > (int64_t(1) << 36))
+    return fail(MUON_ERR_INVALID_ARG, std::string(what) + ": matrix too large (rows, cols <= 2^20, rows*cols <= 2^36)");
+  return MUON_OK;
+}
+
+// Runs the Newton-Schulz phases for every matrix of the plan.
+int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaStream_t s) {
+  const int n = (int)P.shapes.size();
+  const int grid = ds.sms;
+  for (size_t k = 0; k < co.size(); ++k) {
+    const int p = (int)(k & 1);
+    const int first = k == 0 ? 1 : 0;
+    const muon_coeffs_t c = co[k];
+    cudaError_t e;
+    EpiScalars eg{1.0f, 0.0f, first ? 2 : 0, 0};
+    if (P.x_bf16) {
+      e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
+        return launch_gemm_tc(static_cast<GemmProblem*>(P.d_gram[p]), n, P.tiles_gram, eg, ds.d_status, grid, s);
+      });
+    } else {
+      e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
+        return launch_gemm_f32(static_cast<GemmProblemF32*>(P.d_gram[p]), n, P.tiles_gram, eg, grid * 4, s);
+      });
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "gram launch");
+    void* upd;
+    EpiScalars eu;
+    if (c.c != 0.0f) {
+      EpiScalars ep{c.c, c.b, 0, 0};
+      if (P.x_bf16) {
+        e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
+          return launch_gemm_tc(static_cast<GemmProblem*>(P.d_poly), n, P.tiles_poly, ep, ds.d_status, grid, s);
+        });
+      } else {
+        e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
+          return launch_gemm_f32(static_cast<GemmProblemF32*>(P.d_poly), n, P.tiles_poly, ep, grid * 4, s);
+        });
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "poly launch");
+      upd = P.d_updB[p];
+      eu = EpiScalars{1.0f, c.a, first, first};
+    } else {
+      upd = P.d_updA[p];
+      eu = EpiScalars{c.b, c.a, first, first};
+    }
+    if (P.x_bf16) {
+      e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
+        return launch_gemm_tc(static_cast<GemmProblem*>(upd), n, P.tiles_upd, eu, ds.d_status, grid, s);
+      });
+    } else {
+      e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
+        return launch_gemm_f32(static_cast<GemmProblemF32*>(upd), n, P.tiles_upd, eu, grid * 4, s);
+      });
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "update launch");
+  }
+  return MUON_OK;
+}
+
+struct Ranges {   // overlap detection over [begin, end) byte ranges
+  std::vector<std::pair<uintptr_t, uintptr_t>> v;
+  void add(const void* p, size_t bytes) { v.push_back({(uintptr_t)p, (uintptr_t)p + bytes}); }
+  bool overlap() {
+    std::sort(v.begin(), v.end());
+    for (size_t i = 1; i < v.size(); ++i)
+      if (v[i].first < v[i - 1].second) return true;
+    return false;
+  }
+};
+
+}  // namespace
+}  // namespace muon
+
+using namespace muon;
+
+extern "C" {
+
+int muon_version(void) { return 100; }
+
+const char* muon_last_error(void) { return t_err.c_str(); }
+
+int64_t muon_launch_count(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_launches;
+}
+
+int muon_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_prof_on = on != 0;
+  return MUON_OK;
+}
+
+int muon_profile_read(int64_t* launches, double* ms, double* flops, double* exec_flops) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!launches || !ms) return fail(MUON_ERR_INVALID_ARG, "launches and ms must not be NULL");
+  for (int k = 0; k < MUON_KC_COUNT; ++k) {
+    launches[k] = 0;
+    ms[k] = 0.0;
+    if (flops) flops[k] = 0.0;
+    if (exec_flops) exec_flops[k] = 0.0;
+  }
+  int rc = MUON_OK;
+  for (ProfRec& r : g_prof) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess && rc == MUON_OK) rc = cuda_fail(e, "profile event");
+    launches[r.kind] += 1;
+    ms[r.kind] += t;
+    if (flops) flops[r.kind] += r.flops;
+    if (exec_flops) exec_flops[r.kind] += r.exec;
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  return rc;
+}
+
+int muon_check_status(muon_stream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != MUON_OK) return rc;
+  MUON_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  int h[2] = {0, 0};
+  MUON_CUDA(cudaMemcpy(h, ds->d_status, sizeof(h), cudaMemcpyDeviceToHost));
+  MUON_CUDA(cudaMemset(ds->d_status, 0, sizeof(h)));
+  if (h[0] & kStatusTimeout) return fail(MUON_ERR_TIMEOUT, "a kernel wait hit its time limit");
+  if (h[1] != 0) return fail(MUON_WARN_NONFINITE, std::to_string(h[1]) + " chunk(s) held NaN or Inf");
+  return MUON_OK;
+}
+
+int muon_release_workspace(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MUON_OK;
+  auto it = g_dev.find(dev);
+  if (it == g_dev.end()) return MUON_OK;
+  cudaDeviceSynchronize();
+  it->second.plan.reset();
+  return MUON_OK;
+}
+
+int muon_step(int count, float* const* params, const void* const* grads, muon_dtype_t grad_dtype,
+              float* const* momentum, const int64_t* rows, const int64_t* cols, float lr, float mu,
+              int nesterov, float weight_decay, muon_rms_t rms_scale, int steps,
+              const muon_coeffs_t* coeffs, int zero_center, float eps, muon_prec_t prec,
+              muon_stream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  t_err.clear();
+  // ---- validation (no device work before this passes)
+  if (count < 0) return fail(MUON_ERR_INVALID_ARG, "count must be >= 0");
+  if (count > 0 && (!params || !grads || !momentum || !rows || !cols))
+    return fail(MUON_ERR_INVALID_ARG, "params, grads, momentum, rows and cols must not be NULL");
+  if (grad_dtype != MUON_BF16 && grad_dtype != MUON_FP32) return fail(MUON_ERR_INVALID_ARG, "grad_dtype");
+  if (prec != MUON_PREC_BF16 && prec != MUON_PREC_FP32) return fail(MUON_ERR_INVALID_ARG, "prec");
+  if (rms_scale != MUON_RMS_ONE && rms_scale != MUON_RMS_SQRT_MAX1_ROWS_OVER_COLS)
+    return fail(MUON_ERR_INVALID_ARG, "rms_scale");
+  if (!finite_f(lr) || !finite_f(weight_decay)) return fail(MUON_ERR_INVALID_ARG, "lr and weight_decay must be finite");
+  if (!(mu >= 0.0f && mu < 1.0f)) return fail(MUON_ERR_INVALID_ARG, "mu must be in [0, 1)");
+  if (!(eps >= 0.0f) || !finite_f(eps)) return fail(MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  std::vector<muon_coeffs_t> co;
+  int rc = check_coeffs(steps, coeffs, co);
+  if (rc != MUON_OK) return rc;
+  std::vector<int> idx;
+  Ranges written;
+  for (int i = 0; i < count; ++i) {
+    if (!grads[i]) continue;
+    rc = check_shape(rows[i], cols[i], "muon_step");
+    if (rc != MUON_OK) return rc;
+    if (!params[i] || !momentum[i]) return fail(MUON_ERR_INVALID_ARG, "params[i] and momentum[i] must not be NULL");
+    const size_t bytes = (size_t)rows[i] * cols[i] * 4;
+    written.add(params[i], bytes);
+    written.add(momentum[i], bytes);
+    idx.push_back(i);
+  }
+  if (written.overlap()) return fail(MUON_ERR_INVALID_ARG, "params/momentum buffers overlap");
+  if (idx.empty()) return MUON_OK;
+
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != MUON_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<Shape> shapes;
+  for (int i : idx) shapes.push_back({rows[i], cols[i]});
+  const int x_bf16 = prec == MUON_PREC_BF16;
+  Plan* P = nullptr;
+  rc = build_plan(*ds, shapes, x_bf16, &P);
+  if (rc != MUON_OK) return rc;
+  const int n = (int)idx.size();
+  const int g_bf16 = grad_dtype == MUON_BF16;
+  const size_t gsz = g_bf16 ? 2 : 4;
+  std::vector<MatInfo> mats = P->last_uploaded;
+  for (int j = 0; j < n; ++j) {
+    const int i = idx[j];
+    MatInfo& mi = mats[j];
+    mi.p = params[i];
+    mi.g = grads[i];
+    mi.m = momentum[i];
+    mi.xf = (steps & 1) ? P->x1[j] : P->x0[j];
+    mi.rms = rms_scale == MUON_RMS_SQRT_MAX1_ROWS_OVER_COLS
+                 ? (float)std::sqrt(std::max(1.0, (double)rows[i] / (double)cols[i])) : 1.0f;
+    const bool aligned = ((uintptr_t)params[i] % 16 == 0) && ((uintptr_t)momentum[i] % 16 == 0) &&
+                         ((uintptr_t)grads[i] % 16 == 0);
+    mi.vec = (cols[i] % 8 == 0) && aligned ? 1 : 0;
+    (void)gsz;
+  }
+  rc = upload_mats(*P, mats, s);
+  if (rc != MUON_OK) return rc;
+
+  const int ew_grid = ds->sms * 8;
+  cudaError_t e;
+  if (zero_center) {
+    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colsum(P->d_mats, n, P->cs_items, g_bf16, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
+    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colmean(P->d_mats, n, P->cm_items, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "column-mean launch");
+  }
+  e = timed_launch(MUON_KC_PROLOGUE, s, 0, 0, [&] {
+    return launch_prologue(P->d_mats, n, P->n_chunks, g_bf16, x_bf16, 1, mu, nesterov, zero_center,
+                           P->d_partials, ds->d_status, ew_grid, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+  e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(P->d_mats, n, P->d_partials, eps, s); });
+  if (e != cudaSuccess) return cuda_fail(e, "norm launch");
+  rc = run_ns(*ds, *P, co, s);
+  if (rc != MUON_OK) return rc;
+  e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
+    return launch_update(P->d_mats, n, P->n_chunks, x_bf16, lr, 1.0f - lr * weight_decay, steps == 0 ? 1 : 0,
+                         ew_grid, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
+  return MUON_OK;
+}
+
+int muon_ns_orthogonalize(const void* G, muon_dtype_t g_dtype, void* X, muon_dtype_t x_dtype,
+                          int64_t m, int64_t n, int steps, const muon_coeffs_t* coeffs,
+                          int zero_center, float eps, muon_prec_t prec, muon_stream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  t_err.clear();
+  if (!G || !X) return fail(MUON_ERR_INVALID_ARG, "G and X must not be NULL");
+  if (g_dtype != MUON_BF16 && g_dtype != MUON_FP32) return fail(MUON_ERR_INVALID_ARG, "g_dtype");
+  if (x_dtype != MUON_BF16 && x_dtype != MUON_FP32) return fail(MUON_ERR_INVALID_ARG, "x_dtype");
+  if (prec != MUON_PREC_BF16 && prec != MUON_PREC_FP32) return fail(MUON_ERR_INVALID_ARG, "prec");
+  if (!(eps >= 0.0f) || !finite_f(eps)) return fail(MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  int rc = check_shape(m, n, "muon_ns_orthogonalize");
+  if (rc != MUON_OK) return rc;
+  std::vector<muon_coeffs_t> co;
+  rc = check_coeffs(steps, coeffs, co);
+  if (rc != MUON_OK) return rc;
+  Ranges rg;
+  rg.add(G, (size_t)m * n * (g_dtype == MUON_BF16 ? 2 : 4));
+  rg.add(X, (size_t)m * n * (x_dtype == MUON_BF16 ? 2 : 4));
+  if (rg.overlap()) return fail(MUON_ERR_INVALID_ARG, "G and X overlap");
+
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc != MUON_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int x_bf16 = prec == MUON_PREC_BF16;
+  Plan* P = nullptr;
+  rc = build_plan(*ds, {Shape{m, n}}, x_bf16, &P);
+  if (rc != MUON_OK) return rc;
+  std::vector<MatInfo> mats = P->last_uploaded;
+  MatInfo& mi = mats[0];
+  mi.p = static_cast<float*>(X);
+  mi.g = G;
+  mi.m = nullptr;
+  mi.xf = (steps & 1) ? P->x1[0] : P->x0[0];
+  mi.rms = 1.0f;
+  mi.vec = (n % 8 == 0) && ((uintptr_t)G % 16 == 0) && ((uintptr_t)X % 16 == 0) ? 1 : 0;
+  rc = upload_mats(*P, mats, s);
+  if (rc != MUON_OK) return rc;
+  const int g_bf16 = g_dtype == MUON_BF16;
+  const int ew_grid = ds->sms * 8;
+  cudaError_t e;
+  if (zero_center) {
+    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colsum(P->d_mats, 1, P->cs_items, g_bf16, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
+    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colmean(P->d_mats, 1, P->cm_items, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "column-mean launch");
+  }
+  e = timed_launch(MUON_KC_PROLOGUE, s, 0, 0, [&] {
+    return launch_prologue(P->d_mats, 1, P->n_chunks, g_bf16, x_bf16, 0, 0.0f, 0, zero_center,
+                           P->d_partials, ds->d_status, ew_grid, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+  e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(P->d_mats, 1, P->d_partials, eps, s); });
+  if (e != cudaSuccess) return cuda_fail(e, "norm launch");
+  rc = run_ns(*ds, *P, co, s);
+  if (rc != MUON_OK) return rc;
+  e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
+    return launch_output(P->d_mats, 1, P->n_chunks, x_bf16, x_dtype == MUON_BF16, steps == 0 ? 1 : 0,
+                         ew_grid, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "output launch");
+  return MUON_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+// Internal structures shared by the host planner and the device kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace muon {
+
+// Elementwise kernels split every matrix into chunks of this many elements; one CTA owns one
+// chunk at a time and writes one norm partial per chunk.
+constexpr int64_t kChunk = 8192;
+constexpr int kEwThreads = 256;
+
+// Zero-centring work items: column sums over blocks of kCsRows rows x kCsCols columns.
+constexpr int kCsRows = 64;
+constexpr int kCsCols = 256;
+
+// Device status word bits.
+constexpr int kStatusTimeout = 1;
+
+// Per-matrix record read by the elementwise kernels.
+struct MatInfo {
+  float* p;            // fp32 params (muon_step) or output X (orthogonalize), per call
+  const void* g;       // gradient / input, per call
+  float* m;            // fp32 momentum, per call (NULL for orthogonalize)
+  void* x0;            // workspace: U, the unnormalised first iterate (bf16 or fp32)
+  void* xf;            // workspace: final iterate X_steps
+  float* colmean;      // workspace: column means (zero-centring), else NULL
+  float* colpart;      // workspace: column-sum partials (zero-centring), else NULL
+  float* alpha;        // workspace: 1 / (||u||_F + eps)
+  int64_t rows, cols;  // shape of the stored matrix (row-major)
+  int64_t ldx;         // leading dimension of x0 / xf, elements
+  int64_t chunk_begin; // first elementwise chunk of this matrix (prefix over matrices)
+  int64_t cs_begin;    // first column-sum item
+  int64_t cm_begin;    // first column-mean item
+  float rms;           // RMS factor s
+  int vec;             // 1: 16-byte vector path is legal (cols % 8 == 0, aligned pointers)
+};
+
+// One problem of a grouped tensor-core launch:
+//   D = s_acc * (opA . opB^T) + s_c * C,   D: M x N, contraction over K,
+// where opA(i, k) and opB(j, k) are read through TMA from bf16 matrices either K-major
+// (k contiguous) or MN-major (i or j contiguous).
+struct GemmProblem {
+  const CUtensorMap* tma_a;
+  const CUtensorMap* tma_b;
+  __nv_bfloat16* d;
+  const __nv_bfloat16* c;   // addend, may be NULL when s_c == 0
+  const float* alpha;       // per-matrix normalisation 1 / (||u|| + eps)
+  int64_t ldd, ldc;
+  uint32_t M, N, K;
+  uint32_t tiles_m, tiles_n;
+  uint32_t tile_begin;      // prefix sum over the problems of the launch
+  uint32_t n_tiles;
+  uint8_t a_mn, b_mn;       // 1: operand is MN-major
+  uint8_t sym;              // 1: D is symmetric, compute tiles touching the upper triangle
+                            //    and write the strictly-upper part mirrored
+  uint8_t pad;
+};
+
+// fp32 (CUDA-core) problem: same formula, operands addressed by strides.
+struct GemmProblemF32 {
+  const float* a;   // opA(i, k) = a[i * sa_i + k * sa_k]
+  const float* b;   // opB(j, k) = b[j * sb_j + k * sb_k]
+  float* d;
+  const float* c;
+  const float* alpha;
+  int64_t sa_i, sa_k, sb_j, sb_k, ldd, ldc;
+  uint32_t M, N, K;
+  uint32_t tiles_m, tiles_n, tile_begin, n_tiles;
+  uint32_t sym;
+};
+
+// Epilogue scalars of one launch: s_acc = k_acc * alpha^e_acc, s_c = k_c * alpha^e_c.
+struct EpiScalars {
+  float k_acc, k_c;
+  int e_acc, e_c;
+};
+
+// ---- launchers (defined in the .cu files) ----
+cudaError_t launch_colsum(const MatInfo* mats, int nmats, int64_t items, int g_bf16, cudaStream_t s);
+cudaError_t launch_colmean(const MatInfo* mats, int nmats, int64_t items, cudaStream_t s);
+cudaError_t launch_prologue(const MatInfo* mats, int nmats, int64_t chunks, int g_bf16, int x_bf16,
+                            int has_momentum, float mu, int nesterov, int zero_center,
+                            float* partials, int* status, int grid, cudaStream_t s);
+cudaError_t launch_alpha(const MatInfo* mats, int nmats, const float* partials, float eps,
+                         cudaStream_t s);
+cudaError_t launch_update(const MatInfo* mats, int nmats, int64_t chunks, int x_bf16, float lr,
+                          float decay, int scale_by_alpha, int grid, cudaStream_t s);
+cudaError_t launch_output(const MatInfo* mats, int nmats, int64_t chunks, int x_bf16, int out_bf16,
+                          int scale_by_alpha, int grid, cudaStream_t s);
+cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
+                           EpiScalars ep, int* status, int grid, cudaStream_t s);
+cudaError_t launch_gemm_f32(const GemmProblemF32* probs, int nprobs, uint32_t total_tiles,
+                            EpiScalars ep, int grid, cudaStream_t s);
+
+// Tile geometry of the tensor-core kernel.
+constexpr int kTcBM = 128;
+constexpr int kTcBN = 256;
+constexpr int kTcBK = 64;
+// Tile geometry of the fp32 kernel.
+constexpr int kF32BM = 64;
+constexpr int kF32BN = 64;
+
+}  // namespace muon

@@ -1,0 +1,402 @@
+// Newton-Schulz matrix products ("Muon optimizer ..." `newtonschulz5`: A = X X^T,
+// B = b A + c A A, X = a X + B X; "AdamW vs Muon" part 3 writes the same iteration as
+// M_k = a M + b (M M^T) M + c (M M^T)^2 M).
+//
+// One kernel serves all three products. A launch is a list of independent problems (one per
+// matrix of the optimizer step, all at the same iteration and phase), each
+//     D = s_acc * (opA . opB^T) + s_c * C,
+// tiled 128 x 256 and scheduled statically over a persistent grid of one CTA per SM:
+//   warp 0      TMA producer: 64-deep K slices of opA and opB into a 4-stage smem ring
+//               (128-byte swizzle), either K-major boxes or MN-major boxes per operand;
+//   warp 1      tcgen05.mma issuer (one thread): 128 x 256 x 16 bf16 MMAs accumulating in fp32
+//               in tensor memory, two accumulators so the epilogue of one tile overlaps the
+//               MMAs of the next;
+//   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, add s_c * C, round to bf16,
+//               store. For the symmetric products (A = X X^T and A A = A A^T) only tiles that
+//               touch the upper triangle are computed and the strictly-upper part is also
+//               written mirrored.
+// Both orientations of the iterate are read in place: a wide iterate X (m x n) is K-major for
+// X X^T and MN-major as the right operand of B X; a tall stored matrix G (n x m, iterate G^T)
+// is MN-major for G^T G and K-major for G B. So no transposed copies are ever made.
+//
+// Every wait on an mbarrier is bounded: after kTimeoutNs the waiting role sets a shared abort
+// flag and the device status word, the producer waits for its copies in flight, the MMA thread
+// waits for its MMAs, the tensor memory is freed and the CTA returns.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "muon_internal.h"
+#include "ptx.cuh"
+
+namespace muon {
+namespace {
+
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = kTcBM * kTcBK * 2;
+constexpr uint32_t kBBytes = kTcBN * kTcBK * 2;
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kBoxBytes = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 M/N columns
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 2 * kTcBN;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint32_t kGroupM = 8;
+constexpr size_t kBarrierBytes = 256;
+constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
+
+struct Tile {
+  int p;
+  uint32_t bi, bj;
+};
+
+__device__ __forceinline__ Tile decode_tile(const GemmProblem* __restrict__ probs, int nprobs,
+                                            uint32_t t) {
+  int lo = 0, hi = nprobs - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (probs[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
+  }
+  const GemmProblem& P = probs[lo];
+  uint32_t l = t - P.tile_begin;
+  Tile tl;
+  tl.p = lo;
+  if (P.sym) {
+    // row block bi covers rows [128 bi, 128 bi + 128); its first column block touching the
+    // upper triangle is bi / 2 (columns [256 (bi/2), ...)).
+    uint32_t bi = 0;
+    while (true) {
+      const uint32_t cnt = P.tiles_n - bi / 2;
+      if (l < cnt) { tl.bi = bi; tl.bj = bi / 2 + l; break; }
+      l -= cnt;
+      ++bi;
+    }
+  } else {
+    // grouped raster: kGroupM row blocks sweep all column blocks together (L2 reuse)
+    const uint32_t per_group = kGroupM * P.tiles_n;
+    const uint32_t g = l / per_group;
+    const uint32_t first = g * kGroupM;
+    const uint32_t gsize = min(kGroupM, P.tiles_m - first);
+    const uint32_t r = l - g * per_group;
+    tl.bi = first + r % gsize;
+    tl.bj = r / gsize;
+  }
+  return tl;
+}
+
+__device__ __forceinline__ float alpha_pow(float alpha, int e) {
+  float s = 1.0f;
+  for (int i = 0; i < e; ++i) s *= alpha;
+  return s;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    ns_gemm_tc_kernel(const GemmProblem* __restrict__ probs, int nprobs, uint32_t total_tiles,
+                      EpiScalars ep, int* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* tfull = empty + kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* zero_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    *zero_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  bool timed_out = false;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued_parity[kStages];
+      for (int s = 0; s < kStages; ++s) issued_parity[s] = -1;
+      uint32_t stage = 0, phase = 0;
+      for (uint32_t t = blockIdx.x; t < total_tiles && !timed_out; t += gridDim.x) {
+        const Tile tl = decode_tile(probs, nprobs, t);
+        const GemmProblem& P = probs[tl.p];
+        const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
+        const int32_t m0 = (int32_t)(tl.bi * kTcBM), n0 = (int32_t)(tl.bj * kTcBN);
+        for (uint32_t kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+            timed_out = true;
+            break;
+          }
+          uint8_t* a_dst = smem + stage * kStageBytes;
+          uint8_t* b_dst = a_dst + kABytes;
+          const int32_t k0 = (int32_t)(kb * kTcBK);
+          mbar_arrive_expect_tx(&full[stage], kStageBytes);
+          if (!P.a_mn) {
+            tma_load_2d(a_dst, P.tma_a, &full[stage], k0, m0);
+          } else {
+            for (int h = 0; h < kTcBM / 64; ++h)
+              tma_load_2d(a_dst + h * kBoxBytes, P.tma_a, &full[stage], m0 + 64 * h, k0);
+          }
+          if (!P.b_mn) {
+            tma_load_2d(b_dst, P.tma_b, &full[stage], k0, n0);
+          } else {
+            for (int h = 0; h < kTcBN / 64; ++h)
+              tma_load_2d(b_dst + h * kBoxBytes, P.tma_b, &full[stage], n0 + 64 * h, k0);
+          }
+          issued_parity[stage] = (int)phase;
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // copies in flight must land before this CTA's shared memory is released
+      for (int s = 0; s < kStages; ++s)
+        if (issued_parity[s] >= 0)
+          mbar_wait_bounded(&full[s], (uint32_t)issued_parity[s], zero_flag, kTimeoutNs);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      for (uint32_t t = blockIdx.x; t < total_tiles && !timed_out; t += gridDim.x) {
+        const Tile tl = decode_tile(probs, nprobs, t);
+        const GemmProblem& P = probs[tl.p];
+        const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
+        const uint32_t idesc = idesc_bf16_f32(kTcBM, kTcBN, P.a_mn, P.b_mn);
+        const uint32_t a_lbo = P.a_mn ? kBoxBytes : 16u, b_lbo = P.b_mn ? kBoxBytes : 16u;
+        const uint32_t a_kstep = P.a_mn ? 16u * 128u : 32u, b_kstep = P.b_mn ? 16u * 128u : 32u;
+        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+          timed_out = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kTcBN;
+        for (uint32_t kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
+            timed_out = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
+          const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+          for (uint32_t k = 0; k < kTcBK / 16; ++k) {
+            const uint64_t ad = smem_desc_sw128(a_addr + k * a_kstep, a_lbo, 1024);
+            const uint64_t bd = smem_desc_sw128(b_addr + k * b_kstep, b_lbo, 1024);
+            tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (timed_out) break;
+        tc_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // all issued MMAs must finish before the tensor memory is freed
+      tc_commit(drain);
+      mbar_wait_bounded(drain, 0, zero_flag, kTimeoutNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue warps 2..5
+    const uint32_t quarter = (uint32_t)(warp & 3);
+    uint32_t acc = 0, acc_phase = 0;
+    for (uint32_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const Tile tl = decode_tile(probs, nprobs, t);
+      const GemmProblem& P = probs[tl.p];
+      const float alpha = (ep.e_acc | ep.e_c) ? *P.alpha : 1.0f;
+      const float s_acc = ep.k_acc * alpha_pow(alpha, ep.e_acc);
+      const float s_c = ep.k_c * alpha_pow(alpha, ep.e_c);
+      const bool has_c = (P.c != nullptr) && (s_c != 0.0f);
+      // every lane polls; the outcome is made warp-uniform so that the warp stays converged
+      // for the .sync.aligned tensor-memory loads below
+      const bool ok = __all_sync(0xffffffffu,
+                                 mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kTimeoutNs));
+      if (!ok) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      const int64_t row = (int64_t)tl.bi * kTcBM + quarter * 32 + lane;
+      const bool row_ok = row < (int64_t)P.M;
+      const int64_t N = P.N;
+#pragma unroll 1
+      for (int ch = 0; ch < kTcBN / 32; ++ch) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + acc * kTcBN + ch * 32, r);
+        tmem_ld_wait();
+        if (ch == kTcBN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        const int64_t col0 = (int64_t)tl.bj * kTcBN + ch * 32;
+        if (!row_ok || col0 >= N) continue;
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = s_acc * __uint_as_float(r[i]);
+        if (has_c) {
+          const __nv_bfloat16* crow = P.c + row * P.ldc;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int64_t cg = col0 + 8 * g;
+            if (cg + 8 <= N) {
+              const uint4 raw = *reinterpret_cast<const uint4*>(crow + cg);
+              const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float2 f = __bfloat1622float2(h[i]);
+                v[8 * g + 2 * i] += s_c * f.x;
+                v[8 * g + 2 * i + 1] += s_c * f.y;
+              }
+            } else {
+              for (int e = 0; e < 8; ++e)
+                if (cg + e < N) v[8 * g + e] += s_c * __bfloat162float(crow[cg + e]);
+            }
+          }
+        }
+        __nv_bfloat16* drow = P.d + row * P.ldd;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int64_t cg = col0 + 8 * g;
+          if (cg + 8 <= N && (!P.sym || cg >= row)) {
+            uint4 raw;
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[8 * g + 2 * i], v[8 * g + 2 * i + 1]);
+            *reinterpret_cast<uint4*>(drow + cg) = raw;
+          } else {
+            for (int e = 0; e < 8; ++e) {
+              const int64_t col = cg + e;
+              if (col < N && (!P.sym || col >= row)) drow[col] = __float2bfloat16_rn(v[8 * g + e]);
+            }
+          }
+        }
+        if (P.sym) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int64_t col = col0 + i;
+            if (col > row && col < N) P.d[col * P.ldd + row] = __float2bfloat16_rn(v[i]);
+          }
+        }
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  if (timed_out) {
+    *abort_flag = 1;
+    atomicOr(status, kStatusTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ---------------------------------------------------------------- fp32 CUDA-core variant
+constexpr int kF32BK = 16;
+
+__global__ void __launch_bounds__(256)
+    ns_gemm_f32_kernel(const GemmProblemF32* __restrict__ probs, int nprobs, uint32_t total_tiles,
+                       EpiScalars ep) {
+  __shared__ float As[kF32BK][kF32BM + 4];
+  __shared__ float Bs[kF32BK][kF32BN + 4];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  for (uint32_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+    int lo = 0, hi = nprobs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (probs[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
+    }
+    const GemmProblemF32& P = probs[lo];
+    const uint32_t l = t - P.tile_begin;
+    const int64_t i0 = (int64_t)(l / P.tiles_n) * kF32BM, j0 = (int64_t)(l % P.tiles_n) * kF32BN;
+    float acc[4][4] = {};
+    for (int64_t k0 = 0; k0 < P.K; k0 += kF32BK) {
+      for (int e = threadIdx.x; e < kF32BK * kF32BM; e += blockDim.x) {
+        const int kk = e / kF32BM, ii = e % kF32BM;
+        const int64_t gi = i0 + ii, gk = k0 + kk;
+        As[kk][ii] = (gi < P.M && gk < P.K) ? P.a[gi * P.sa_i + gk * P.sa_k] : 0.0f;
+        const int64_t gj = j0 + ii;
+        Bs[kk][ii] = (gj < P.N && gk < P.K) ? P.b[gj * P.sb_j + gk * P.sb_k] : 0.0f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < kF32BK; ++kk) {
+        float a[4], b[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          a[x] = As[kk][ty * 4 + x];
+          b[x] = Bs[kk][tx * 4 + x];
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(a[x], b[y], acc[x][y]);
+      }
+      __syncthreads();
+    }
+    const float alpha = (ep.e_acc | ep.e_c) ? *P.alpha : 1.0f;
+    const float s_acc = ep.k_acc * alpha_pow(alpha, ep.e_acc);
+    const float s_c = ep.k_c * alpha_pow(alpha, ep.e_c);
+    for (int x = 0; x < 4; ++x) {
+      const int64_t gi = i0 + ty * 4 + x;
+      if (gi >= P.M) continue;
+      for (int y = 0; y < 4; ++y) {
+        const int64_t gj = j0 + tx * 4 + y;
+        if (gj >= P.N) continue;
+        float v = s_acc * acc[x][y];
+        if (P.c != nullptr && s_c != 0.0f) v += s_c * P.c[gi * P.ldc + gj];
+        P.d[gi * P.ldd + gj] = v;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
+                           EpiScalars ep, int* status, int grid, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  if (total_tiles == 0) return cudaSuccess;
+  if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
+  ns_gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_f32(const GemmProblemF32* probs, int nprobs, uint32_t total_tiles,
+                            EpiScalars ep, int grid, cudaStream_t s) {
+  if (total_tiles == 0) return cudaSuccess;
+  if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
+  ns_gemm_f32_kernel<<<grid, 256, 0, s>>>(probs, nprobs, total_tiles, ep);
+  return cudaGetLastError();
+}
+
+size_t gemm_tc_smem_bytes() { return kSmemBytes; }
+
+}  // namespace muon
