@@ -134,6 +134,37 @@ MUON_API int muon_step(int count, float* const* params, const void* const* grads
               const muon_coeffs_t* coeffs, int zero_center, float eps, muon_prec_t prec,
               muon_stream_t stream);
 
+/*
+ * Newton-Schulz orthogonalisation of one matrix that allocates nothing.
+ * (No counterpart in the pages: this is an interface concern, not part of the method.)
+ *
+ * For callers that cannot allocate device memory while they run: for example a plugin or
+ * custom-call hook whose host framework owns all allocations and forbids cudaMalloc inside its
+ * execution callback, or a service that reserves its memory at start-up and allocates nothing
+ * afterwards. muon_ns_orthogonalize allocates its workspace with cudaMalloc on first use; this
+ * call instead works in a fixed scratch area compiled into the library (a __device__ array of
+ * about 12.1 MiB, reserved on every device that loads the library and held until the process
+ * exits), and calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   G, g_dtype, X, x_dtype, m, n, steps, coeffs, eps   as for muon_ns_orthogonalize
+ *           (bf16 working precision; no zero-centring).
+ *   status  optional device pointer to 2 ints owned by the caller, or NULL. Kernels set
+ *           bit 0 of status[0] when a wait hits its time limit (the result is then invalid)
+ *           and add to status[1] the number of 8192-element chunks that held NaN or Inf; the
+ *           caller clears it. With NULL these go to a word in the scratch area, cleared by
+ *           every call, that the caller cannot read.
+ * Limits: min(m, n) <= 1024 and m * round_up(n, 8) <= 2097152 elements; larger matrices are
+ * rejected with MUON_ERR_INVALID_ARG (use muon_ns_orthogonalize).
+ * The first call on a device sets that device up (it looks up the scratch address); make that
+ * first call before any stream capture. All calls share the one scratch area and overwrite it:
+ * calls must be ordered on the GPU (one stream, or synchronised by the caller); calls that
+ * overlap on the GPU race. Returns MUON_OK or a negative error code.
+ */
+MUON_API int muon_ns_orthogonalize_noalloc(const void* G, muon_dtype_t g_dtype, void* X,
+                                           muon_dtype_t x_dtype, int64_t m, int64_t n, int steps,
+                                           const muon_coeffs_t* coeffs, float eps, int* status,
+                                           muon_stream_t stream);
+
 /* Message describing the last error returned on the calling thread ("" if none). The pointer
  * stays valid until the next call on that thread. */
 MUON_API const char* muon_last_error(void);

@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmuon.so")
-SOURCES = ["api.cu", "elementwise.cu", "ns_gemm.cu"]
+SOURCES = ["api.cu", "elementwise.cu", "ns_gemm.cu", "noalloc.cu"]
 HEADERS = ["muon_internal.h", "ptx.cuh"]
 
 NVCC_FLAGS = [

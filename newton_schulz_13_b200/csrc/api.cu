@@ -557,6 +557,16 @@ struct Ranges {   // overlap detection over [begin, end) byte ranges
 };
 
 }  // namespace
+
+// Hooks for the no-allocation entry point (noalloc.cu): its error message and launch count go
+// through the same per-thread message and counter as every other call.
+void set_error_message(const std::string& msg) { t_err = msg; }
+
+void note_launches(int64_t n) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_launches += n;
+}
+
 }  // namespace muon
 
 using namespace muon;
