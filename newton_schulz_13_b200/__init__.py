@@ -100,6 +100,8 @@ def _coeff_array(steps: int, coeffs: Optional[Sequence[Tuple[float, float, float
 def _stream_handle(stream) -> Optional[int]:
     import torch
     if stream is None:
+        if not torch.cuda.is_available():
+            return None   # the library reports the missing device itself
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
