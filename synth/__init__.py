@@ -256,6 +256,12 @@ WORKLOADS = {
         zero_center=False, eps=1e-7, n_steps=1, layer_size=7),
 }
 
+# One layer of the Llama-8B set (7 matrices, 2.2e8 elements): a few GB on the device, still
+# larger than L2, used for detailed kernel profiles.
+WORKLOADS["llama8b_layer"] = Workload(**{**WORKLOADS["llama8b"].__dict__, "name": "llama8b_layer",
+                                         "description": "one layer of the Llama-8B hidden-weight set",
+                                         "shapes": WORKLOADS["llama8b"].shapes[:7]})
+
 # The eight-plus-two coefficient schedule (eight quintic iterations, then two
 # with (2, -1.5, 0.5)), exercised on the GPT-2-small shapes.
 HYBRID = [(3.445, -4.7750, 2.0315)] * 8 + [(2.0, -1.5, 0.5)] * 2

@@ -1,0 +1,170 @@
+"""Whole-workload parity: every matrix of each workload goes through one muon_step launch sequence
+(the same launches bench.py times), and sampled matrices are compared with the fp64 oracle run
+on its own trajectory from the same seeded inputs. No value produced by the CUDA path is ever fed
+to the oracle.
+
+Per step and per sampled matrix:
+  O (recovered from the device's own parameters before and after the step) <= 3e-2 (bf16 mode),
+  momentum <= 1e-6, parameters <= k * 1e-3 after k steps (the per-step bound, accumulated: the two
+  trajectories differ only through the O error of each step).
+For the Llama-8B shapes too large for the oracle (4096 x 4096, 14336 x 4096, 4096 x 14336) the
+checks are properties of the method that hold at any size:
+  - momentum element by element (the oracle with zero Newton-Schulz iterations);
+  - O X0^T (wide) or X0^T O (tall) is symmetric, since O = r(X0 X0^T) X0 for a polynomial r;
+  - on the top singular triplets (sigma, u, v) of X0, O v = phi(sigma) u, with phi the scalar map;
+  - ||O||_F^2 = sum_i phi(sigma_i)^2 over all singular values of X0.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.gpu_util import TOL_M, TOL_O_BF16, TOL_O_FP32, TOL_P, StepCase, host64, rel, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def scalar_map(x, coeffs):
+    x = np.asarray(x, dtype=np.float64).copy()
+    for a, b, c in coeffs:
+        x = a * x + b * x ** 3 + c * x ** 5
+    return x
+
+
+def run_and_check(case: StepCase, n_steps: int, prec: str = "bf16", tol_o: float = TOL_O_BF16):
+    wl = case.wl
+    decay = np.float64(np.float32(1.0 - np.float32(wl.lr) * np.float32(wl.weight_decay)))
+    lr32 = np.float64(np.float32(wl.lr))
+    worst = {"O": 0.0, "m": 0.0, "p": 0.0}
+    for k in range(n_steps):
+        p_prev = {j: host64(case.params[j]) for j in case.sample}
+        _, O_ref = case.step(k, prec=prec)
+        torch.cuda.synchronize()
+        for j in case.sample:
+            p_new = host64(case.params[j])
+            assert np.all(np.isfinite(p_new)), j
+            O_gpu = (p_prev[j] * decay - p_new) / (lr32 * case.rms(j))
+            e_o = rel(O_gpu, O_ref[j])
+            e_m = rel(host64(case.momentum[j]), case.o_mom[j])
+            e_p = rel(p_new, case.o_params[j])
+            worst["O"], worst["m"], worst["p"] = max(worst["O"], e_o), max(worst["m"], e_m), max(worst["p"], e_p)
+            assert e_o <= tol_o, (k, j, "O", e_o)
+            assert e_m <= TOL_M, (k, j, "momentum", e_m)
+            assert e_p <= (k + 1) * TOL_P, (k, j, "params", e_p)
+    import newton_schulz_13_b200 as ns
+    assert ns.check_status() == ns.OK
+    print(f"{wl.name} {prec}: worst O {worst['O']:.2e}, momentum {worst['m']:.2e}, params {worst['p']:.2e}")
+    return worst
+
+
+def test_cubic_zero_center_12():
+    wl = synth.WORKLOADS["cubic_zero_center_12"]
+    run_and_check(StepCase(wl, sample=list(range(12))), wl.n_steps)
+
+
+def test_cubic_zero_center_12_fp32_mode():
+    wl = synth.WORKLOADS["cubic_zero_center_12"]
+    run_and_check(StepCase(wl, sample=[0, 6, 11]), wl.n_steps, prec="fp32", tol_o=TOL_O_FP32)
+
+
+def test_single_256x512_fp32_mode():
+    wl = synth.WORKLOADS["single_256x512"]
+    run_and_check(StepCase(wl, sample=[0]), 1, prec="fp32", tol_o=TOL_O_FP32)
+
+
+def test_gpt2_small_ten_steps():
+    wl = synth.WORKLOADS["gpt2_small"]
+    # layer 0's square and tall (transposed path) matrices, and the last layer's square one
+    run_and_check(StepCase(wl, sample=[1, 3, 45], device_fill=True), wl.n_steps)
+
+
+def test_gpt2_small_hybrid_schedule():
+    wl = synth.WORKLOADS["gpt2_small"]
+    case = StepCase(wl, sample=[0, 2], device_fill=True)
+    decay = np.float64(np.float32(1.0 - np.float32(wl.lr) * np.float32(wl.weight_decay)))
+    p_prev = {j: host64(case.params[j]) for j in case.sample}
+    _, O_ref = case.step(0, coeffs=synth.HYBRID)
+    for j in case.sample:
+        O_gpu = (p_prev[j] * decay - host64(case.params[j])) / np.float64(np.float32(wl.lr))
+        assert rel(O_gpu, O_ref[j]) <= TOL_O_BF16
+
+
+def test_mamba_24_three_steps():
+    wl = synth.WORKLOADS["mamba_24"]
+    # layer 0 (all four shapes, two of them tall) and the last layer's thin projections
+    run_and_check(StepCase(wl, sample=[0, 1, 2, 3, 93, 94], device_fill=True), wl.n_steps)
+
+
+# ----------------------------------------------------------------------------- Llama-8B, full size
+def _top_triplets(X: np.ndarray, k: int = 6, iters: int = 80, seed: int = 0):
+    """Top-k singular triplets of X by block power iteration with a final Rayleigh-Ritz step."""
+    rng = np.random.default_rng(seed)
+    V = np.linalg.qr(rng.standard_normal((X.shape[1], 2 * k)))[0]
+    for _ in range(iters):
+        V = np.linalg.qr(X.T @ (X @ V))[0]
+    XV = X @ V
+    Uh, s, Wt = np.linalg.svd(XV, full_matrices=False)
+    Vr = V @ Wt.T
+    return Uh[:, :k], s[:k], Vr[:, :k]
+
+
+def test_llama8b_full_size():
+    import newton_schulz_13_b200 as ns
+    wl = synth.WORKLOADS["llama8b"]
+    exact = [1, 2, 218]                  # Wk, Wv of layer 0; Wk of layer 31 (1024 x 4096)
+    props = [0, 4, 6, 220]               # Wq, gate (tall), down (wide) of layer 0; Wo of layer 31
+    case = StepCase(wl, sample=exact + props, device_fill=True)
+    # the oracle's full step only for the matrices it finishes in seconds
+    big = {j: case.o_params.pop(j) for j in props}
+    case.sample = exact
+    p_prev = {j: host64(case.params[j]) for j in exact + props}
+    g, O_ref = case.step(0)
+    torch.cuda.synchronize()
+    assert ns.check_status() == ns.OK
+    decay = np.float64(np.float32(1.0 - np.float32(wl.lr) * np.float32(wl.weight_decay)))
+    lr32 = np.float64(np.float32(wl.lr))
+    for j in exact:
+        p_new = host64(case.params[j])
+        O_gpu = (p_prev[j] * decay - p_new) / (lr32 * case.rms(j))
+        assert rel(O_gpu, O_ref[j]) <= TOL_O_BF16, j
+        assert rel(p_new, case.o_params[j]) <= TOL_P, j
+        assert rel(host64(case.momentum[j]), case.o_mom[j]) <= TOL_M, j
+    rng = np.random.default_rng(7)
+    for j in props:
+        r, c = wl.shapes[j]
+        gj = host64(g[j])
+        # momentum and the normalised update X0 from the oracle with zero iterations
+        m_ref = np.zeros((r, c))
+        X0 = oracle.muon_step([big[j].copy()], [gj], [m_ref], lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov,
+                              weight_decay=wl.weight_decay, rms_mode=wl.rms_scale, coeffs=[],
+                              zero_center=False, eps=wl.eps, want_O=True)[0]
+        assert rel(host64(case.momentum[j]), m_ref) <= TOL_M, j
+        p_new = host64(case.params[j])
+        O = (p_prev[j] * decay - p_new) / (lr32 * case.rms(j))
+        assert np.all(np.isfinite(O))
+        tall = r > c
+        # symmetry of O X0^T (wide) or X0^T O (tall), probed with random vectors
+        R = rng.standard_normal((r if not tall else c, 16))
+        if not tall:
+            M = (O.T @ R).T @ (X0.T @ R)
+        else:
+            M = (O @ R).T @ (X0 @ R)
+        asym = np.linalg.norm(M - M.T) / np.linalg.norm(M)
+        assert asym <= 0.05, (j, "asymmetry", asym)
+        # the scalar map on the top singular triplets
+        Xo = X0 if not tall else X0.T
+        Oo = O if not tall else O.T
+        U, s, V = _top_triplets(Xo)
+        phi = scalar_map(s, wl.coeffs)
+        for i in range(len(s)):
+            resid = np.linalg.norm(Xo.T @ U[:, i] - s[i] * V[:, i]) / s[i]
+            if resid > 1e-3:
+                continue   # not converged (clustered values): skip this one
+            err = np.linalg.norm(Oo @ V[:, i] - phi[i] * U[:, i]) / phi[i]
+            assert err <= 0.05, (j, i, "triplet", err)
+        # Frobenius norm against the whole spectrum
+        sig2 = np.linalg.eigvalsh(Xo @ Xo.T)
+        want = np.sqrt(np.sum(scalar_map(np.sqrt(np.clip(sig2, 0, None)), wl.coeffs) ** 2))
+        got = np.linalg.norm(O)
+        assert abs(got / want - 1.0) <= 0.02, (j, "frobenius", got, want)
