@@ -29,8 +29,6 @@
 
 namespace muon {
 
-size_t gemm_tc_smem_bytes();
-
 namespace {
 
 thread_local std::string t_err;
@@ -112,8 +110,8 @@ struct Shape {
   bool operator==(const Shape& o) const { return r == o.r && c == o.c; }
 };
 
-struct BufMaps {   // three TMA views of one bf16 buffer
-  int k128 = -1, k256 = -1, mn64 = -1;
+struct BufMaps {   // TMA views of one bf16 buffer: operand loads and the epilogue's store view
+  int k128 = -1, k256 = -1, mn64 = -1, st32 = -1;
 };
 
 struct Plan {
@@ -156,6 +154,7 @@ struct DeviceState {
   int* d_status = nullptr;  // [0] flags, [1] non-finite count
   int sms = 0;
   int cc_major = 0;
+  int pair_capacity = 0;   // resident CTA pairs of the paired tensor-core kernel
 };
 
 std::map<int, DeviceState> g_dev;
@@ -173,6 +172,7 @@ int device_state(DeviceState** out) {
   }
   if (ds.cc_major != 10)
     return fail(MUON_ERR_UNSUPPORTED, "this library runs on sm_100 (B200) devices only");
+  if (ds.pair_capacity == 0) ds.pair_capacity = gemm_tc_pair_capacity(ds.sms);
   if (!ds.d_status) {
     MUON_CUDA(cudaMalloc(&ds.d_status, 2 * sizeof(int)));
     MUON_CUDA(cudaMemset(ds.d_status, 0, 2 * sizeof(int)));
@@ -227,7 +227,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   const size_t o_alpha = off; off = align_up(off + (size_t)n * 4, AL);
   const size_t o_part = off; off = align_up(off + (size_t)chunks * 4, AL);
   const size_t o_mats = off; off = align_up(off + (size_t)n * sizeof(MatInfo), AL);
-  const int maps_per = 12;
+  const int maps_per = 16;   // 4 buffers x 4 views
   const size_t o_maps = off;
   if (x_bf16) off = align_up(off + (size_t)n * maps_per * sizeof(CUtensorMap), AL);
   const size_t prob_sz = x_bf16 ? sizeof(GemmProblem) : sizeof(GemmProblemF32);
@@ -260,11 +260,11 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   }
 
   // ---- grouped problems
+  // CTA-pair tiles are 256 x 256; a symmetric m x m product computes the T (T + 1) / 2 tiles on or
+  // above the diagonal, T = ceil(m / 256).
   auto sym_tiles = [](int64_t m) {
-    const int64_t tm = ceil_div(m, kTcBM), tn = ceil_div(m, kTcBN);
-    int64_t t = 0;
-    for (int64_t bi = 0; bi < tm; ++bi) t += tn - bi / 2;
-    return t;
+    const int64_t t = ceil_div(m, kTcPairBM);
+    return t * (t + 1) / 2;
   };
   if (x_bf16) {
     PFN_encodeTiled_t encode = get_encode();
@@ -272,18 +272,22 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     std::vector<CUtensorMap> maps((size_t)n * maps_per);
     CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(W + o_maps);
     int bad = 0;
-    auto make3 = [&](int j, int slot, void* base, int64_t rows, int64_t cols, int64_t ld) {
+    // views: 64-wide K-major boxes of 128 or 256 rows and 64 x 64 MN-major boxes (128-byte
+    // swizzle, operand loads), and 32 x 32 boxes with the 64-byte swizzle (epilogue stores)
+    auto make4 = [&](int j, int slot, void* base, int64_t rows, int64_t cols, int64_t ld) {
       BufMaps bm;
-      const int boxes[3] = {kTcBM, kTcBN, 64};
-      int* dst[3] = {&bm.k128, &bm.k256, &bm.mn64};
-      for (int b = 0; b < 3; ++b) {
-        const int idx = j * maps_per + slot * 3 + b;
+      const cuuint32_t bx[4] = {64u, 64u, 64u, 32u}, by[4] = {(cuuint32_t)kTcBM, (cuuint32_t)kTcBN, 64u, 32u};
+      const CUtensorMapSwizzle sw[4] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_128B,
+                                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_64B};
+      int* dst[4] = {&bm.k128, &bm.k256, &bm.mn64, &bm.st32};
+      for (int b = 0; b < 4; ++b) {
+        const int idx = j * maps_per + slot * 4 + b;
         cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
         cuuint64_t gstride[1] = {(cuuint64_t)(ld * 2)};
-        cuuint32_t box[2] = {64u, (cuuint32_t)boxes[b]};
+        cuuint32_t box[2] = {bx[b], by[b]};
         cuuint32_t estr[2] = {1u, 1u};
         CUresult r = encode(&maps[idx], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, gdim, gstride, box,
-                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw[b],
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) bad = (int)r;
         *dst[b] = idx;
@@ -295,21 +299,22 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     for (int j = 0; j < n; ++j) {
       const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c), nn = std::max(r, c);
       const bool tall = r > c;
-      BufMaps mx[2] = {make3(j, 0, P->x0[j], r, c, P->ldx[j]), make3(j, 1, P->x1[j], r, c, P->ldx[j])};
-      BufMaps mA = make3(j, 2, P->A[j], m, m, P->ldm[j]);
-      BufMaps mB = make3(j, 3, P->B[j], m, m, P->ldm[j]);
+      BufMaps mx[2] = {make4(j, 0, P->x0[j], r, c, P->ldx[j]), make4(j, 1, P->x1[j], r, c, P->ldx[j])};
+      BufMaps mA = make4(j, 2, P->A[j], m, m, P->ldm[j]);
+      BufMaps mB = make4(j, 3, P->B[j], m, m, P->ldm[j]);
       auto M_ = [&](int idx) { return d_maps + idx; };
       for (int p = 0; p < 2; ++p) {
         GemmProblem g{};
         g.tma_a = M_(tall ? mx[p].mn64 : mx[p].k128);
-        g.tma_b = M_(tall ? mx[p].mn64 : mx[p].k256);
+        g.tma_b = M_(tall ? mx[p].mn64 : mx[p].k128);
         g.a_mn = g.b_mn = tall ? 1 : 0;
         g.d = static_cast<__nv_bfloat16*>(P->A[j]);
         g.ldd = P->ldm[j];
+        g.tma_d = M_(mA.st32);
         g.alpha = P->alpha[j];
         g.M = g.N = (uint32_t)m;
         g.K = (uint32_t)nn;
-        g.tiles_m = (uint32_t)ceil_div(m, kTcBM);
+        g.tiles_m = (uint32_t)ceil_div(m, kTcPairBM);
         g.tiles_n = (uint32_t)ceil_div(m, kTcBN);
         g.sym = 1;
         g.n_tiles = (uint32_t)sym_tiles(m);
@@ -325,15 +330,14 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
             u.tma_b = M_(mx[p].mn64); u.b_mn = 1;
           } else {
             u.tma_a = M_(mx[p].k128); u.a_mn = 0;
-            u.tma_b = M_(mS.k256); u.b_mn = 0;
+            u.tma_b = M_(mS.k128); u.b_mn = 0;
           }
           u.d = static_cast<__nv_bfloat16*>(p == 0 ? P->x1[j] : P->x0[j]);
           u.ldd = P->ldx[j];
-          u.c = static_cast<const __nv_bfloat16*>(p == 0 ? P->x0[j] : P->x1[j]);
-          u.ldc = P->ldx[j];
+          u.tma_d = M_(mx[1 - p].st32);
           u.alpha = P->alpha[j];
           u.M = (uint32_t)r; u.N = (uint32_t)c; u.K = (uint32_t)m;
-          u.tiles_m = (uint32_t)ceil_div(r, kTcBM);
+          u.tiles_m = (uint32_t)ceil_div(r, kTcPairBM);
           u.tiles_n = (uint32_t)ceil_div(c, kTcBN);
           u.n_tiles = u.tiles_m * u.tiles_n;
           u.tile_begin = tu;
@@ -341,12 +345,15 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
         }
       }
       GemmProblem q{};
-      q.tma_a = M_(mA.k128); q.tma_b = M_(mA.k256);
+      // B = c A A + b A (+ a I on the tensor-core path): A is symmetric, so A A = A A^T
+      q.tma_a = M_(mA.k128); q.tma_b = M_(mA.k128);
       q.d = static_cast<__nv_bfloat16*>(P->B[j]); q.ldd = P->ldm[j];
       q.c = static_cast<const __nv_bfloat16*>(P->A[j]); q.ldc = P->ldm[j];
+      q.tma_d = M_(mB.st32);
+      q.tma_c = M_(mA.st32);
       q.alpha = P->alpha[j];
       q.M = q.N = q.K = (uint32_t)m;
-      q.tiles_m = (uint32_t)ceil_div(m, kTcBM); q.tiles_n = (uint32_t)ceil_div(m, kTcBN);
+      q.tiles_m = (uint32_t)ceil_div(m, kTcPairBM); q.tiles_n = (uint32_t)ceil_div(m, kTcBN);
       q.sym = 1;
       q.n_tiles = (uint32_t)sym_tiles(m);
       q.tile_begin = tp;
@@ -357,7 +364,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       P->fl_gram += 2.0 * m * m * nn;
       P->fl_poly += 2.0 * m * m * m;
       P->fl_upd += 2.0 * m * m * nn;
-      const double tile_fl = 2.0 * kTcBM * kTcBN;
+      const double tile_fl = 2.0 * kTcPairBM * kTcBN;
       P->ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kTcBK) * kTcBK);
       P->ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
       P->ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
@@ -500,10 +507,15 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
     const int first = k == 0 ? 1 : 0;
     const muon_coeffs_t c = co[k];
     cudaError_t e;
-    EpiScalars eg{1.0f, 0.0f, first ? 2 : 0, 0};
+    // fp32 path: gram A = alpha^2k X X^T, poly B = c A A + b A, update X' = alpha^k (a X + B X)
+    //   (c = 0: X' = alpha^k (a X + b A X)).
+    // bf16 path: the a X term is folded into the left operand of the update, rounding once:
+    //   poly B = c A A + b A + a I (c = 0: gram A = b alpha^2k X X^T + a I), update X' = alpha^k B X.
+    EpiScalars eg{1.0f, 0.0f, first ? 2 : 0, 0, 0.0f};
+    if (P.x_bf16 && c.c == 0.0f) eg = EpiScalars{c.b, 0.0f, first ? 2 : 0, 0, c.a};
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
-        return launch_gemm_tc(static_cast<GemmProblem*>(P.d_gram[p]), n, P.tiles_gram, eg, ds.d_status, grid, s);
+        return launch_gemm_tc_pair(static_cast<GemmProblem*>(P.d_gram[p]), n, P.tiles_gram, eg, ds.d_status, ds.pair_capacity, s);
       });
     } else {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
@@ -514,10 +526,10 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
     void* upd;
     EpiScalars eu;
     if (c.c != 0.0f) {
-      EpiScalars ep{c.c, c.b, 0, 0};
+      EpiScalars ep{c.c, c.b, 0, 0, P.x_bf16 ? c.a : 0.0f};
       if (P.x_bf16) {
         e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
-          return launch_gemm_tc(static_cast<GemmProblem*>(P.d_poly), n, P.tiles_poly, ep, ds.d_status, grid, s);
+          return launch_gemm_tc_pair(static_cast<GemmProblem*>(P.d_poly), n, P.tiles_poly, ep, ds.d_status, ds.pair_capacity, s);
         });
       } else {
         e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
@@ -526,14 +538,14 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
       }
       if (e != cudaSuccess) return cuda_fail(e, "poly launch");
       upd = P.d_updB[p];
-      eu = EpiScalars{1.0f, c.a, first, first};
+      eu = P.x_bf16 ? EpiScalars{1.0f, 0.0f, first, 0, 0.0f} : EpiScalars{1.0f, c.a, first, first, 0.0f};
     } else {
       upd = P.d_updA[p];
-      eu = EpiScalars{c.b, c.a, first, first};
+      eu = P.x_bf16 ? EpiScalars{1.0f, 0.0f, first, 0, 0.0f} : EpiScalars{c.b, c.a, first, first, 0.0f};
     }
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
-        return launch_gemm_tc(static_cast<GemmProblem*>(upd), n, P.tiles_upd, eu, ds.d_status, grid, s);
+        return launch_gemm_tc_pair(static_cast<GemmProblem*>(upd), n, P.tiles_upd, eu, ds.d_status, ds.pair_capacity, s);
       });
     } else {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {

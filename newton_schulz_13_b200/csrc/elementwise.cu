@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(kCsCols) colmean_kernel(const MatInfo* __restr
 
 // ---------------------------------------------------------------- prologue
 template <bool G_BF16, bool X_BF16>
-__global__ void __launch_bounds__(kEwThreads) prologue_kernel(const MatInfo* __restrict__ mats, int nmats,
+__global__ void __launch_bounds__(kEwThreads, 4) prologue_kernel(const MatInfo* __restrict__ mats, int nmats,
                                                               int64_t nchunks, int has_m, float mu,
                                                               int nesterov, int zc,
                                                               float* __restrict__ partials,
@@ -145,7 +145,51 @@ __global__ void __launch_bounds__(kEwThreads) prologue_kernel(const MatInfo* __r
     const int64_t e1 = min(n_el, e0 + kChunk);
     float sq = 0.f;
     int bad = 0;
-    if (mi.vec) {
+    if (mi.vec && e1 - e0 == kChunk) {
+      // a full chunk: each thread owns kGroups groups of 8 elements and handles them kBatch at a
+      // time, issuing all loads of a batch before any arithmetic (more bytes in flight per thread)
+      constexpr int kGroups = (int)(kChunk / (8 * kEwThreads));
+      constexpr int kBatch = 2;
+#pragma unroll
+      for (int b0 = 0; b0 < kGroups; b0 += kBatch) {
+        float g[kBatch][8], m[kBatch][8];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int64_t e = e0 + 8 * ((int64_t)threadIdx.x + (int64_t)(b0 + q) * kEwThreads);
+          load8<G_BF16>(mi.g, e, g[q]);
+          if (has_m) load8<false>(mi.m, e, m[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int64_t e = e0 + 8 * ((int64_t)threadIdx.x + (int64_t)(b0 + q) * kEwThreads);
+          const int64_t row = e / mi.cols, col = e - row * mi.cols;
+          float u[8];
+          if (zc) {
+            const float4* cm = reinterpret_cast<const float4*>(mi.colmean + col);
+            const float4 c0 = cm[0], c1 = cm[1];
+            g[q][0] -= c0.x; g[q][1] -= c0.y; g[q][2] -= c0.z; g[q][3] -= c0.w;
+            g[q][4] -= c1.x; g[q][5] -= c1.y; g[q][6] -= c1.z; g[q][7] -= c1.w;
+          }
+          if (has_m) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              m[q][i] = mu * m[q][i] + one_m_mu * g[q][i];
+              u[i] = nesterov ? mu * m[q][i] + one_m_mu * g[q][i] : m[q][i];
+            }
+            store8<false>(mi.m, e, m[q]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = g[q][i];
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            sq += u[i] * u[i];
+            bad |= !isfinite(u[i]);
+          }
+          store8<X_BF16>(mi.x0, row * mi.ldx + col, u);
+        }
+      }
+    } else if (mi.vec) {
       for (int64_t e = e0 + 8 * (int64_t)threadIdx.x; e < e1; e += 8 * (int64_t)blockDim.x) {
         const int64_t row = e / mi.cols, col = e - row * mi.cols;
         float g[8], u[8];
@@ -217,7 +261,7 @@ __global__ void __launch_bounds__(256) alpha_kernel(const MatInfo* __restrict__ 
 
 // ---------------------------------------------------------------- update / output
 template <bool X_BF16>
-__global__ void __launch_bounds__(kEwThreads) update_kernel(const MatInfo* __restrict__ mats, int nmats,
+__global__ void __launch_bounds__(kEwThreads, 4) update_kernel(const MatInfo* __restrict__ mats, int nmats,
                                                             int64_t nchunks, float lr, float decay,
                                                             int scale_by_alpha) {
   for (int64_t chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
@@ -227,7 +271,29 @@ __global__ void __launch_bounds__(kEwThreads) update_kernel(const MatInfo* __res
     const int64_t e0 = (chunk - mi.chunk_begin) * kChunk;
     const int64_t e1 = min(n_el, e0 + kChunk);
     const float step = lr * mi.rms * (scale_by_alpha ? *mi.alpha : 1.0f);
-    if (mi.vec) {
+    if (mi.vec && e1 - e0 == kChunk) {
+      // a full chunk: loads of kBatch groups are issued before their arithmetic
+      constexpr int kGroups = (int)(kChunk / (8 * kEwThreads));
+      constexpr int kBatch = 2;
+#pragma unroll
+      for (int b0 = 0; b0 < kGroups; b0 += kBatch) {
+        float o[kBatch][8], p[kBatch][8];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int64_t e = e0 + 8 * ((int64_t)threadIdx.x + (int64_t)(b0 + q) * kEwThreads);
+          const int64_t row = e / mi.cols, col = e - row * mi.cols;
+          load8<X_BF16>(mi.xf, row * mi.ldx + col, o[q]);
+          load8<false>(mi.p, e, p[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int64_t e = e0 + 8 * ((int64_t)threadIdx.x + (int64_t)(b0 + q) * kEwThreads);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) p[q][i] = p[q][i] * decay - step * o[q][i];
+          store8<false>(mi.p, e, p[q]);
+        }
+      }
+    } else if (mi.vec) {
       for (int64_t e = e0 + 8 * (int64_t)threadIdx.x; e < e1; e += 8 * (int64_t)blockDim.x) {
         const int64_t row = e / mi.cols, col = e - row * mi.cols;
         float o[8], p[8];

@@ -46,8 +46,10 @@ struct MatInfo {
 struct GemmProblem {
   const CUtensorMap* tma_a;
   const CUtensorMap* tma_b;
+  const CUtensorMap* tma_d;   // CTA-pair kernel: TMA store view (32 x 32 boxes) of d
+  const CUtensorMap* tma_c;   // CTA-pair kernel: TMA load view (32 x 32 boxes) of the addend, or NULL
   __nv_bfloat16* d;
-  const __nv_bfloat16* c;   // addend, may be NULL when s_c == 0
+  const __nv_bfloat16* c;   // single-CTA kernel: addend, may be NULL when s_c == 0
   const float* alpha;       // per-matrix normalisation 1 / (||u|| + eps)
   int64_t ldd, ldc;
   uint32_t M, N, K;
@@ -73,10 +75,12 @@ struct GemmProblemF32 {
   uint32_t sym;
 };
 
-// Epilogue scalars of one launch: s_acc = k_acc * alpha^e_acc, s_c = k_c * alpha^e_c.
+// Epilogue scalars of one launch: D = k_acc alpha^e_acc acc + k_c alpha^e_c C + diag I
+// (diag is applied by the CTA-pair kernel only, on symmetric outputs).
 struct EpiScalars {
   float k_acc, k_c;
   int e_acc, e_c;
+  float diag;
 };
 
 // ---- launchers (defined in the .cu files) ----
@@ -93,11 +97,16 @@ cudaError_t launch_output(const MatInfo* mats, int nmats, int64_t chunks, int x_
                           int scale_by_alpha, int grid, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                            EpiScalars ep, int* status, int grid, cudaStream_t s);
+cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
+                                EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
+int gemm_tc_pair_capacity(int sms);
 cudaError_t launch_gemm_f32(const GemmProblemF32* probs, int nprobs, uint32_t total_tiles,
                             EpiScalars ep, int grid, cudaStream_t s);
 
-// Tile geometry of the tensor-core kernel.
+// Tile geometry of the tensor-core kernel: single-CTA tiles are kTcBM x kTcBN, CTA-pair tiles
+// kTcPairBM x kTcBN; K advances kTcBK per pipeline stage.
 constexpr int kTcBM = 128;
+constexpr int kTcPairBM = 256;
 constexpr int kTcBN = 256;
 constexpr int kTcBK = 64;
 // Tile geometry of the fp32 kernel.

@@ -31,23 +31,45 @@
 namespace muon {
 namespace {
 
-constexpr int kStages = 4;
-constexpr uint32_t kABytes = kTcBM * kTcBK * 2;
-constexpr uint32_t kBBytes = kTcBN * kTcBK * 2;
-constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kBoxBytes = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 M/N columns
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 2 * kTcBN;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kGroupM = 8;
-constexpr size_t kBarrierBytes = 256;
-constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + kBarrierBytes;
+
+// Geometry of the two variants. Each CTA owns 128 accumulator rows x 256 columns (two
+// accumulators = all 512 tensor-memory columns).
+//   single CTA: output tile 128 x 256, the CTA loads 128 rows of opA and 256 rows of opB.
+//   CTA pair:   output tile 256 x 256; each CTA loads its 128 rows of opA and 128 of the 256 opB
+//               rows, the even CTA issues 256 x 256 x 16 MMAs that read both CTAs' stages.
+template <bool PAIR>
+struct TcCfg {
+  static constexpr int kTileM = PAIR ? 256 : 128;
+  static constexpr int kTileN = 256;
+  static constexpr int kBRows = PAIR ? 128 : 256;
+  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr uint32_t kABytes = 128 * kTcBK * 2;
+  static constexpr uint32_t kBBytes = kBRows * kTcBK * 2;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kTmemCols = 2 * kTileN;
+  static constexpr uint32_t kEpiArrivals = PAIR ? 8 : 4;
+  // CTA pair: per epilogue warp two staging sets (direct + mirrored 32 x 32 bf16 sub-tiles)
+  static constexpr uint32_t kStagingPerWarp = 2 * 2 * 2048;
+  static constexpr uint32_t kStagingBytes = PAIR ? 4 * kStagingPerWarp : 0;
+  static constexpr size_t kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 256;
+};
+
+// Byte offset of 16-byte chunk j of row r in a 32-row x 64-byte staging box laid out with the
+// 64-byte swizzle the TMA store expects (chunk index XOR bits 1-2 of the row).
+__device__ __forceinline__ uint32_t sw64_chunk(uint32_t r, uint32_t j) {
+  return r * 64u + ((j ^ ((r >> 1) & 3u)) << 4);
+}
 
 struct Tile {
   int p;
   uint32_t bi, bj;
 };
 
+template <int TILE_M, int TILE_N>
 __device__ __forceinline__ Tile decode_tile(const GemmProblem* __restrict__ probs, int nprobs,
                                             uint32_t t) {
   int lo = 0, hi = nprobs - 1;
@@ -60,12 +82,13 @@ __device__ __forceinline__ Tile decode_tile(const GemmProblem* __restrict__ prob
   Tile tl;
   tl.p = lo;
   if (P.sym) {
-    // row block bi covers rows [128 bi, 128 bi + 128); its first column block touching the
-    // upper triangle is bi / 2 (columns [256 (bi/2), ...)).
+    // row block bi covers rows [TILE_M bi, TILE_M (bi + 1)); its first column block touching the
+    // upper triangle is (TILE_M bi) / TILE_N.
     uint32_t bi = 0;
     while (true) {
-      const uint32_t cnt = P.tiles_n - bi / 2;
-      if (l < cnt) { tl.bi = bi; tl.bj = bi / 2 + l; break; }
+      const uint32_t first = (bi * TILE_M) / TILE_N;
+      const uint32_t cnt = P.tiles_n - first;
+      if (l < cnt) { tl.bi = bi; tl.bj = first + l; break; }
       l -= cnt;
       ++bi;
     }
@@ -88,98 +111,134 @@ __device__ __forceinline__ float alpha_pow(float alpha, int e) {
   return s;
 }
 
+template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     ns_gemm_tc_kernel(const GemmProblem* __restrict__ probs, int nprobs, uint32_t total_tiles,
                       EpiScalars ep, int* __restrict__ status) {
+  using C = TcCfg<PAIR>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
-  uint64_t* empty = full + kStages;
-  uint64_t* tfull = empty + kStages;
+  uint8_t* staging = smem + C::kStages * C::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::kStagingBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* drain = tempty + 2;                       // followed by 4 addend-load barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* zero_flag = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;      // 0: the CTA that issues the MMAs
+  const bool leader = rank == 0;
+  const uint32_t unit = PAIR ? blockIdx.x / 2 : blockIdx.x;  // pair (or CTA) index
+  const uint32_t n_units = PAIR ? gridDim.x / 2 : gridDim.x;
+
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], C::kEpiArrivals);
     }
     mbar_init(drain, 1);
+    for (int w = 0; w < 4; ++w) mbar_init(drain + 1 + w, 1);
     *abort_flag = 0;
     *zero_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // the peer may signal the even CTA's barriers from now on
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   bool timed_out = false;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (every CTA)
     if (lane == 0) {
-      int issued_parity[kStages];
-      for (int s = 0; s < kStages; ++s) issued_parity[s] = -1;
+      int issued_parity[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) issued_parity[s] = -1;
       uint32_t stage = 0, phase = 0;
-      for (uint32_t t = blockIdx.x; t < total_tiles && !timed_out; t += gridDim.x) {
-        const Tile tl = decode_tile(probs, nprobs, t);
+      for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
+        const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
         const GemmProblem& P = probs[tl.p];
         const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
-        const int32_t m0 = (int32_t)(tl.bi * kTcBM), n0 = (int32_t)(tl.bj * kTcBN);
+        const int32_t a_row0 = (int32_t)(tl.bi * C::kTileM + rank * 128);
+        const int32_t b_row0 = (int32_t)(tl.bj * C::kTileN + rank * C::kBRows);
         for (uint32_t kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
             timed_out = true;
             break;
           }
-          uint8_t* a_dst = smem + stage * kStageBytes;
-          uint8_t* b_dst = a_dst + kABytes;
+          uint8_t* a_dst = smem + stage * C::kStageBytes;
+          uint8_t* b_dst = a_dst + C::kABytes;
           const int32_t k0 = (int32_t)(kb * kTcBK);
-          mbar_arrive_expect_tx(&full[stage], kStageBytes);
-          if (!P.a_mn) {
-            tma_load_2d(a_dst, P.tma_a, &full[stage], k0, m0);
+          if constexpr (PAIR) {
+            // both halves of the pair count on the even CTA's barrier
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+            if (!P.a_mn) {
+              tma_load_2d_pair(a_dst, P.tma_a, bar, k0, a_row0);
+            } else {
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d_pair(a_dst + h * kBoxBytes, P.tma_a, bar, a_row0 + 64 * h, k0);
+            }
+            if (!P.b_mn) {
+              tma_load_2d_pair(b_dst, P.tma_b, bar, k0, b_row0);
+            } else {
+              for (int h = 0; h < C::kBRows / 64; ++h)
+                tma_load_2d_pair(b_dst + h * kBoxBytes, P.tma_b, bar, b_row0 + 64 * h, k0);
+            }
           } else {
-            for (int h = 0; h < kTcBM / 64; ++h)
-              tma_load_2d(a_dst + h * kBoxBytes, P.tma_a, &full[stage], m0 + 64 * h, k0);
-          }
-          if (!P.b_mn) {
-            tma_load_2d(b_dst, P.tma_b, &full[stage], k0, n0);
-          } else {
-            for (int h = 0; h < kTcBN / 64; ++h)
-              tma_load_2d(b_dst + h * kBoxBytes, P.tma_b, &full[stage], n0 + 64 * h, k0);
+            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            if (!P.a_mn) {
+              tma_load_2d(a_dst, P.tma_a, &full[stage], k0, a_row0);
+            } else {
+              for (int h = 0; h < 2; ++h)
+                tma_load_2d(a_dst + h * kBoxBytes, P.tma_a, &full[stage], a_row0 + 64 * h, k0);
+            }
+            if (!P.b_mn) {
+              tma_load_2d(b_dst, P.tma_b, &full[stage], k0, b_row0);
+            } else {
+              for (int h = 0; h < C::kBRows / 64; ++h)
+                tma_load_2d(b_dst + h * kBoxBytes, P.tma_b, &full[stage], b_row0 + 64 * h, k0);
+            }
           }
           issued_parity[stage] = (int)phase;
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      // copies in flight must land before this CTA's shared memory is released
-      for (int s = 0; s < kStages; ++s)
-        if (issued_parity[s] >= 0)
-          mbar_wait_bounded(&full[s], (uint32_t)issued_parity[s], zero_flag, kTimeoutNs);
+      // copies in flight must land before this CTA's shared memory is released (the even CTA's
+      // barriers also count the odd CTA's copies)
+      if (leader)
+        for (int s = 0; s < C::kStages; ++s)
+          if (issued_parity[s] >= 0)
+            mbar_wait_bounded(&full[s], (uint32_t)issued_parity[s], zero_flag, kTimeoutNs);
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      for (uint32_t t = blockIdx.x; t < total_tiles && !timed_out; t += gridDim.x) {
-        const Tile tl = decode_tile(probs, nprobs, t);
+      for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
+        const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
         const GemmProblem& P = probs[tl.p];
         const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
-        const uint32_t idesc = idesc_bf16_f32(kTcBM, kTcBN, P.a_mn, P.b_mn);
+        const uint32_t idesc = idesc_bf16_f32(C::kTileM, C::kTileN, P.a_mn, P.b_mn);
         const uint32_t a_lbo = P.a_mn ? kBoxBytes : 16u, b_lbo = P.b_mn ? kBoxBytes : 16u;
         const uint32_t a_kstep = P.a_mn ? 16u * 128u : 32u, b_kstep = P.b_mn ? 16u * 128u : 32u;
         if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
@@ -187,39 +246,154 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kTcBN;
+        const uint32_t d_tmem = tmem_base + acc * C::kTileN;
         for (uint32_t kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
             timed_out = true;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * kStageBytes);
-          const uint32_t b_addr = a_addr + kABytes;
+          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b_addr = a_addr + C::kABytes;
 #pragma unroll
           for (uint32_t k = 0; k < kTcBK / 16; ++k) {
             const uint64_t ad = smem_desc_sw128(a_addr + k * a_kstep, a_lbo, 1024);
             const uint64_t bd = smem_desc_sw128(b_addr + k * b_kstep, b_lbo, 1024);
-            tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0u);
+            if constexpr (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0u);
+            else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0u);
           }
-          tc_commit(&empty[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+          if constexpr (PAIR) tc_commit_pair_mc(&empty[stage], 0x3);
+          else tc_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
         if (timed_out) break;
-        tc_commit(&tfull[acc]);
+        if constexpr (PAIR) tc_commit_pair_mc(&tfull[acc], 0x3);
+        else tc_commit(&tfull[acc]);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       // all issued MMAs must finish before the tensor memory is freed
-      tc_commit(drain);
+      if constexpr (PAIR) tc_commit_pair(drain);
+      else tc_commit(drain);
       mbar_wait_bounded(drain, 0, zero_flag, kTimeoutNs);
     }
+    __syncwarp();
+  } else if constexpr (PAIR) {
+    // ------------------------------------------------------------ epilogue warps 2..5 (pair)
+    // Each warp owns 32 accumulator rows. Per 32-column chunk it forms
+    //   D = k_acc alpha^e acc + k_c C + diag I
+    // in fp32, rounds to bf16, stages the 32 x 32 sub-tile in shared memory (64-byte swizzle) and
+    // writes it with a TMA store. The addend sub-tile C, when there is one, arrives by TMA in the
+    // same staging buffer first. For symmetric outputs, sub-tiles strictly above the diagonal are
+    // also staged transposed and stored at the mirrored position, sub-tiles strictly below are
+    // skipped (their mirror writes them) and diagonal sub-tiles are stored whole. Rows and
+    // columns past the matrix are clipped by the TMA store.
+    const uint32_t quarter = (uint32_t)(warp & 3);
+    uint8_t* stg = staging + (uint32_t)(warp - 2) * C::kStagingPerWarp;
+    uint64_t* cbar = drain + 1 + (warp - 2);    // this warp's addend-load barrier
+    uint32_t set = 0, cphase = 0;
+    uint32_t acc = 0, acc_phase = 0;
+    for (uint32_t t = unit; t < total_tiles; t += n_units) {
+      const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
+      const GemmProblem& P = probs[tl.p];
+      const float alpha = ep.e_acc ? *P.alpha : 1.0f;
+      const float s1 = ep.k_acc * alpha_pow(alpha, ep.e_acc);
+      const bool has_c = P.tma_c != nullptr && ep.k_c != 0.0f;
+      const bool ok = __all_sync(0xffffffffu,
+                                 mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kTimeoutNs));
+      if (!ok) {
+        timed_out = true;
+        break;
+      }
+      tc_fence_after();
+      const int32_t r0 = (int32_t)(tl.bi * C::kTileM + rank * 128 + quarter * 32);
+#pragma unroll 1
+      for (int ch = 0; ch < C::kTileN / 32; ++ch) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + acc * C::kTileN + ch * 32, r);
+        tmem_ld_wait();
+        if (ch == C::kTileN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        }
+        const int32_t c0 = (int32_t)(tl.bj * C::kTileN + ch * 32);
+        if (r0 >= (int32_t)P.M || c0 >= (int32_t)P.N) continue;        // fully clipped
+        if (P.sym && c0 + 32 <= r0) continue;                            // mirrored elsewhere
+        const bool diag_blk = P.sym && c0 == r0;
+        const bool mirror = P.sym && c0 >= r0 + 32;
+        uint8_t* direct = stg + set * 4096u;
+        uint8_t* mirr = direct + 2048u;
+        if (lane == 0) bulk_wait_group_read<1>();   // the store issued from this set has read it
+        __syncwarp();
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = s1 * __uint_as_float(r[i]);
+        if (has_c) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(cbar, 2048u);
+            tma_load_2d(direct, P.tma_c, cbar, c0, r0);
+          }
+          const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(cbar, cphase, abort_flag, kTimeoutNs));
+          cphase ^= 1u;
+          if (!got) {
+            timed_out = true;
+            break;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 raw = *reinterpret_cast<const uint4*>(direct + sw64_chunk((uint32_t)lane, (uint32_t)j));
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(h[i]);
+              v[8 * j + 2 * i] += ep.k_c * f.x;
+              v[8 * j + 2 * i + 1] += ep.k_c * f.y;
+            }
+          }
+          __syncwarp();   // every lane has read its addend row before the buffer is overwritten
+        }
+        if (diag_blk) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i == lane) v[i] += ep.diag;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 raw;
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[8 * j + 2 * i], v[8 * j + 2 * i + 1]);
+          *reinterpret_cast<uint4*>(direct + sw64_chunk((uint32_t)lane, (uint32_t)j)) = raw;
+        }
+        if (mirror) {
+          // element (row lane, column i) goes to row i, column lane of the transposed box
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const uint32_t off = sw64_chunk((uint32_t)i, (uint32_t)lane >> 3) + ((uint32_t)lane & 7u) * 2u;
+            *reinterpret_cast<__nv_bfloat16*>(mirr + off) = __float2bfloat16_rn(v[i]);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(P.tma_d, direct, c0, r0);
+          if (mirror) tma_store_2d(P.tma_d, mirr, r0, c0);
+          bulk_commit_group();
+        }
+        set ^= 1u;
+      }
+      if (timed_out) break;
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (lane == 0) bulk_wait_group_all();
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue warps 2..5
     const uint32_t quarter = (uint32_t)(warp & 3);
     uint32_t acc = 0, acc_phase = 0;
-    for (uint32_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const Tile tl = decode_tile(probs, nprobs, t);
+    for (uint32_t t = unit; t < total_tiles; t += n_units) {
+      const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
       const GemmProblem& P = probs[tl.p];
       const float alpha = (ep.e_acc | ep.e_c) ? *P.alpha : 1.0f;
       const float s_acc = ep.k_acc * alpha_pow(alpha, ep.e_acc);
@@ -234,21 +408,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int64_t row = (int64_t)tl.bi * kTcBM + quarter * 32 + lane;
+      const int64_t row = (int64_t)tl.bi * C::kTileM + rank * 128 + quarter * 32 + lane;
       const bool row_ok = row < (int64_t)P.M;
       const int64_t N = P.N;
 #pragma unroll 1
-      for (int ch = 0; ch < kTcBN / 32; ++ch) {
+      for (int ch = 0; ch < C::kTileN / 32; ++ch) {
         uint32_t r[32];
         __syncwarp();
-        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + acc * kTcBN + ch * 32, r);
+        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + acc * C::kTileN + ch * 32, r);
         tmem_ld_wait();
-        if (ch == kTcBN / 32 - 1) {
+        if (ch == C::kTileN / 32 - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
-        const int64_t col0 = (int64_t)tl.bj * kTcBN + ch * 32;
+        const int64_t col0 = (int64_t)tl.bj * C::kTileN + ch * 32;
         if (!row_ok || col0 >= N) continue;
         float v[32];
 #pragma unroll
@@ -308,8 +482,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // the pair leaves together: no CTA exits while its partner may still signal its barriers or
+  // (even CTA) write its tensor memory
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+  if (warp == 1) {
+    if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
+  }
 }
 
 // ---------------------------------------------------------------- fp32 CUDA-core variant
@@ -376,17 +556,71 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                            EpiScalars ep, int* status, int grid, cudaStream_t s) {
+  using C = TcCfg<false>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   if (total_tiles == 0) return cudaSuccess;
   if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
-  ns_gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status);
+  ns_gemm_tc_kernel<false><<<grid, kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
+                                EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
+  using C = TcCfg<true>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  if (total_tiles == 0) return cudaSuccess;
+  const uint32_t pairs = (uint32_t)max_pairs < total_tiles ? (uint32_t)max_pairs : total_tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ns_gemm_tc_kernel<true>, probs, nprobs, total_tiles, ep, status);
+}
+
+// Largest number of CTA pairs of the paired kernel that can be resident at once.
+int gemm_tc_pair_capacity(int sms) {
+  using C = TcCfg<true>;
+  cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)C::kSmemBytes);
+  if (e != cudaSuccess) return sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, ns_gemm_tc_kernel<true>, &cfg);
+  if (e != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return sms / 2;
+  }
+  return n;
 }
 
 cudaError_t launch_gemm_f32(const GemmProblemF32* probs, int nprobs, uint32_t total_tiles,
@@ -397,6 +631,5 @@ cudaError_t launch_gemm_f32(const GemmProblemF32* probs, int nprobs, uint32_t to
   return cudaGetLastError();
 }
 
-size_t gemm_tc_smem_bytes() { return kSmemBytes; }
 
 }  // namespace muon
