@@ -264,7 +264,10 @@ def run_ours(args, world, rank, local):
     traffic = recorded_traffic()
     elements = wl.elements()
     gbytes = 1 if wl.grad_dtype == "bf16" else 2
-    ew_bytes = elements * ((2 * gbytes + 4 + 4 + 2) + (2 + 4 + 4))
+    # prologue: grad + m read + m write + bf16 U write; a separate epilogue kernel (used when the
+    # parameter update is not fused into the last Newton-Schulz launch): bf16 O + p read + p write
+    fused_update = prof["epilogue"][0] == 0
+    ew_bytes = elements * ((2 * gbytes + 4 + 4 + 2) + (0 if fused_update else (2 + 4 + 4)))
     ew_ms = prof["prologue"][1] + prof["epilogue"][1] + prof["norm"][1] + prof["center"][1]
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     ew_achieved = ew_bytes * args.steps / (ew_ms * 1e-3) / 1e9 if ew_ms > 0 else None
@@ -294,7 +297,9 @@ def run_ours(args, world, rank, local):
                                  "frac": (ew_achieved / hbm_peak) if ew_achieved else None,
                                  "bytes_per_step": ew_bytes,
                                  "bytes_definition": "per element: grad + m read + m write + bf16 U write "
-                                                     "(prologue), bf16 O read + p read + p write (epilogue)",
+                                                     "(prologue)" + ("; the parameter update is fused into the "
+                                                     "last Newton-Schulz launch" if fused_update else
+                                                     ", bf16 O read + p read + p write (epilogue)"),
                                  "ms_per_step": ew_ms / args.steps},
         "kernels_ms_per_step": {k: v[1] / args.steps for k, v in prof.items()},
         "gpu_launches": launches,

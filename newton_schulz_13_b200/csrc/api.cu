@@ -141,8 +141,18 @@ struct Plan {
   MatInfo* h_pinned = nullptr;
   cudaEvent_t upload_done = nullptr;
   bool uploaded_once = false;
+  // fused last update (tensor-core path): host copies of the update problems, and the per-call
+  // table of the last iteration's update problems with TMA views of the caller's parameters
+  std::vector<GemmProblem> h_upd[2][2];    // [operand: 0 B, 1 A][parity]
+  CUtensorMap* d_pmaps = nullptr;
+  GemmProblem* d_fused = nullptr;
+  uint8_t* h_fused_pinned = nullptr;
+  cudaEvent_t fused_done = nullptr;
+  std::vector<uint8_t> fused_key;
 
   ~Plan() {
+    if (fused_done) cudaEventDestroy(fused_done);
+    if (h_fused_pinned) cudaFreeHost(h_fused_pinned);
     if (upload_done) cudaEventDestroy(upload_done);
     if (h_pinned) cudaFreeHost(h_pinned);
     if (ws) cudaFree(ws);
@@ -233,6 +243,10 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   const size_t prob_sz = x_bf16 ? sizeof(GemmProblem) : sizeof(GemmProblemF32);
   size_t o_prob[7];
   for (int k = 0; k < 7; ++k) { o_prob[k] = off; off = align_up(off + (size_t)n * prob_sz, AL); }
+  const size_t o_pmaps = off;
+  if (x_bf16) off = align_up(off + (size_t)n * sizeof(CUtensorMap), AL);
+  const size_t o_fused = off;
+  if (x_bf16) off = align_up(off + (size_t)n * sizeof(GemmProblem), AL);
   P->ws_bytes = off;
 
   cudaError_t e = cudaMalloc(&P->ws, P->ws_bytes);
@@ -380,6 +394,12 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       MUON_CUDA(cudaMemcpy(*dsts[k], lists[k]->data(), lists[k]->size() * sizeof(GemmProblem),
                            cudaMemcpyHostToDevice));
     }
+    P->h_upd[0][0] = updB[0]; P->h_upd[0][1] = updB[1];
+    P->h_upd[1][0] = updA[0]; P->h_upd[1][1] = updA[1];
+    P->d_pmaps = reinterpret_cast<CUtensorMap*>(W + o_pmaps);
+    P->d_fused = reinterpret_cast<GemmProblem*>(W + o_fused);
+    MUON_CUDA(cudaMallocHost(&P->h_fused_pinned, (size_t)n * (sizeof(CUtensorMap) + sizeof(GemmProblem))));
+    MUON_CUDA(cudaEventCreateWithFlags(&P->fused_done, cudaEventDisableTiming));
   } else {
     std::vector<GemmProblemF32> gram[2], poly, updB[2], updA[2];
     uint32_t tg = 0, tp = 0, tu = 0;
@@ -476,6 +496,56 @@ int upload_mats(Plan& P, std::vector<MatInfo>& mats, cudaStream_t s) {
   return MUON_OK;
 }
 
+// Per-call table of the last Newton-Schulz update with the parameter update fused into its
+// epilogue: the plan's update problems plus TMA views (32 x 32 fp32 boxes, 128-byte swizzle) of
+// the caller's parameter matrices. Rebuilt and uploaded only when the parameters, the RMS factors
+// or the last iteration's operand and parity change. Returns NULL when a parameter matrix cannot
+// be viewed by TMA (row length not a multiple of 4 floats, or a base not 16-byte aligned); the
+// step then uses the separate update kernel.
+const GemmProblem* fused_table(Plan& P, float* const* params, const std::vector<int>& idx,
+                               const std::vector<float>& rms, int which, int parity, cudaStream_t s,
+                               int* rc) {
+  *rc = MUON_OK;
+  const int n = (int)P.shapes.size();
+  for (int j = 0; j < n; ++j)
+    if (P.shapes[j].c % 4 != 0 || (uintptr_t)params[idx[j]] % 16 != 0) return nullptr;
+  std::vector<uint8_t> key(sizeof(void*) * n + sizeof(float) * n + 2 * sizeof(int));
+  uint8_t* k = key.data();
+  for (int j = 0; j < n; ++j) { std::memcpy(k, &params[idx[j]], sizeof(void*)); k += sizeof(void*); }
+  std::memcpy(k, rms.data(), sizeof(float) * n); k += sizeof(float) * n;
+  std::memcpy(k, &which, sizeof(int)); k += sizeof(int);
+  std::memcpy(k, &parity, sizeof(int));
+  if (key == P.fused_key) return P.d_fused;
+  PFN_encodeTiled_t encode = get_encode();
+  if (!encode) return nullptr;
+  std::vector<CUtensorMap> maps(n);
+  std::vector<GemmProblem> probs = P.h_upd[which][parity];
+  for (int j = 0; j < n; ++j) {
+    cuuint64_t gdim[2] = {(cuuint64_t)P.shapes[j].c, (cuuint64_t)P.shapes[j].r};
+    cuuint64_t gstride[1] = {(cuuint64_t)(P.shapes[j].c * 4)};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = encode(&maps[j], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, params[idx[j]], gdim, gstride, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return nullptr;
+    probs[j].tma_p = P.d_pmaps + j;
+    probs[j].rms = rms[j];
+  }
+  cudaError_t e = cudaEventSynchronize(P.fused_done);
+  if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table event"); return nullptr; }
+  std::memcpy(P.h_fused_pinned, maps.data(), n * sizeof(CUtensorMap));
+  std::memcpy(P.h_fused_pinned + n * sizeof(CUtensorMap), probs.data(), n * sizeof(GemmProblem));
+  e = cudaMemcpyAsync(P.d_pmaps, P.h_fused_pinned, n * sizeof(CUtensorMap), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(P.d_fused, P.h_fused_pinned + n * sizeof(CUtensorMap), n * sizeof(GemmProblem),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaEventRecord(P.fused_done, s);
+  if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table upload"); return nullptr; }
+  P.fused_key = key;
+  return P.d_fused;
+}
+
 bool finite_f(float x) { return std::isfinite(x); }
 
 int check_coeffs(int steps, const muon_coeffs_t* coeffs, std::vector<muon_coeffs_t>& out) {
@@ -499,7 +569,8 @@ int check_shape(int64_t r, int64_t c, const char* what) {
 }
 
 // Runs the Newton-Schulz phases for every matrix of the plan.
-int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaStream_t s) {
+int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaStream_t s,
+           const GemmProblem* fused_last = nullptr, float lr = 0.0f, float decay = 1.0f) {
   const int n = (int)P.shapes.size();
   const int grid = ds.sms;
   for (size_t k = 0; k < co.size(); ++k) {
@@ -542,6 +613,12 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
     } else {
       upd = P.d_updA[p];
       eu = P.x_bf16 ? EpiScalars{1.0f, 0.0f, first, 0, 0.0f} : EpiScalars{c.b, c.a, first, first, 0.0f};
+    }
+    if (fused_last && k + 1 == co.size()) {
+      upd = const_cast<GemmProblem*>(fused_last);
+      eu.lr = lr;
+      eu.decay = decay;
+      eu.fused = 1;
     }
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
@@ -717,6 +794,14 @@ int muon_step(int count, float* const* params, const void* const* grads, muon_dt
   }
   rc = upload_mats(*P, mats, s);
   if (rc != MUON_OK) return rc;
+  const GemmProblem* fused = nullptr;
+  if (x_bf16 && steps > 0) {
+    std::vector<float> rms(n);
+    for (int j = 0; j < n; ++j) rms[j] = mats[j].rms;
+    const int which = co.back().c != 0.0f ? 0 : 1;
+    fused = fused_table(*P, params, idx, rms, which, (steps - 1) & 1, s, &rc);
+    if (rc != MUON_OK) return rc;
+  }
 
   const int ew_grid = ds->sms * 8;
   cudaError_t e;
@@ -733,8 +818,9 @@ int muon_step(int count, float* const* params, const void* const* grads, muon_dt
   if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
   e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(P->d_mats, n, P->d_partials, eps, s); });
   if (e != cudaSuccess) return cuda_fail(e, "norm launch");
-  rc = run_ns(*ds, *P, co, s);
+  rc = run_ns(*ds, *P, co, s, fused, lr, 1.0f - lr * weight_decay);
   if (rc != MUON_OK) return rc;
+  if (fused) return MUON_OK;   // the last update GEMM already wrote the parameters
   e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
     return launch_update(P->d_mats, n, P->n_chunks, x_bf16, lr, 1.0f - lr * weight_decay, steps == 0 ? 1 : 0,
                          ew_grid, s);

@@ -48,6 +48,7 @@ struct GemmProblem {
   const CUtensorMap* tma_b;
   const CUtensorMap* tma_d;   // CTA-pair kernel: TMA store view (32 x 32 boxes) of d
   const CUtensorMap* tma_c;   // CTA-pair kernel: TMA load view (32 x 32 boxes) of the addend, or NULL
+  const CUtensorMap* tma_p;   // CTA-pair kernel, fused last update: fp32 parameters (32 x 32 boxes)
   __nv_bfloat16* d;
   const __nv_bfloat16* c;   // single-CTA kernel: addend, may be NULL when s_c == 0
   const float* alpha;       // per-matrix normalisation 1 / (||u|| + eps)
@@ -56,6 +57,7 @@ struct GemmProblem {
   uint32_t tiles_m, tiles_n;
   uint32_t tile_begin;      // prefix sum over the problems of the launch
   uint32_t n_tiles;
+  float rms;                // fused last update: RMS factor s of this matrix
   uint8_t a_mn, b_mn;       // 1: operand is MN-major
   uint8_t sym;              // 1: D is symmetric, compute tiles touching the upper triangle
                             //    and write the strictly-upper part mirrored
@@ -76,11 +78,15 @@ struct GemmProblemF32 {
 };
 
 // Epilogue scalars of one launch: D = k_acc alpha^e_acc acc + k_c alpha^e_c C + diag I
-// (diag is applied by the CTA-pair kernel only, on symmetric outputs).
+// (diag is applied by the CTA-pair kernel only, on symmetric outputs). With fused set (CTA-pair
+// kernel, last Newton-Schulz update), O = k_acc alpha^e_acc acc is not stored; instead the
+// parameters become p (1 - lr wd) - lr s O, with decay = 1 - lr wd and s = rms of the problem.
 struct EpiScalars {
   float k_acc, k_c;
   int e_acc, e_c;
   float diag;
+  float lr, decay;
+  int fused;
 };
 
 // ---- launchers (defined in the .cu files) ----

@@ -326,6 +326,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* mirr = direct + 2048u;
         if (lane == 0) bulk_wait_group_read<1>();   // the store issued from this set has read it
         __syncwarp();
+        if (ep.fused) {
+          // last update: the whole 4 KB set holds the 32 x 32 fp32 parameter sub-tile (128-byte
+          // swizzle); O stays in fp32 and is never stored
+          if (lane == 0) {
+            mbar_arrive_expect_tx(cbar, 4096u);
+            tma_load_2d(direct, P.tma_p, cbar, c0, r0);
+          }
+          const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(cbar, cphase, abort_flag, kTimeoutNs));
+          cphase ^= 1u;
+          if (!got) {
+            timed_out = true;
+            break;
+          }
+          const float step = ep.lr * P.rms * s1;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4* q = reinterpret_cast<float4*>(direct + (uint32_t)lane * 128u +
+                                                  ((((uint32_t)j) ^ ((uint32_t)lane & 7u)) << 4));
+            float4 pv = *q;
+            pv.x = pv.x * ep.decay - step * __uint_as_float(r[4 * j + 0]);
+            pv.y = pv.y * ep.decay - step * __uint_as_float(r[4 * j + 1]);
+            pv.z = pv.z * ep.decay - step * __uint_as_float(r[4 * j + 2]);
+            pv.w = pv.w * ep.decay - step * __uint_as_float(r[4 * j + 3]);
+            *q = pv;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(P.tma_p, direct, c0, r0);
+            bulk_commit_group();
+          }
+          set ^= 1u;
+          continue;
+        }
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = s1 * __uint_as_float(r[i]);
