@@ -43,6 +43,10 @@ def load(path: Optional[str] = None):
                                      ctypes.POINTER(dp), i64p, i64p, ctypes.c_double, ctypes.c_double,
                                      ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int, dp,
                                      ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.POINTER(dp)]
+    lib.oracle_adamw_step.restype = ctypes.c_int
+    lib.oracle_adamw_step.argtypes = [ctypes.c_int, ctypes.POINTER(dp), ctypes.POINTER(dp), ctypes.POINTER(dp),
+                                      ctypes.POINTER(dp), i64p, ctypes.c_int64, ctypes.c_double, ctypes.c_double,
+                                      ctypes.c_double, ctypes.c_double, ctypes.c_double]
     if path is None:
         _lib = lib
     return lib
@@ -97,3 +101,25 @@ def muon_step(params: List[np.ndarray], grads: List[Optional[np.ndarray]], momen
     if rc != 0:
         raise ValueError("oracle_muon_step rejected its arguments")
     return outs
+
+
+def adamw_step(params: List[np.ndarray], grads: List[Optional[np.ndarray]], exp_avg: List[np.ndarray],
+               exp_avg_sq: List[np.ndarray], step: int, lr: float, beta1: float, beta2: float, eps: float,
+               weight_decay: float, lib=None) -> None:
+    """One AdamW step in fp64 (any shapes; arrays are updated in place). `step` is the step count
+    after this step (1 for the first)."""
+    lib = lib or load()
+    n = len(params)
+    for a in list(params) + list(exp_avg) + list(exp_avg_sq):
+        assert a.dtype == np.float64 and a.flags["C_CONTIGUOUS"]
+    g64 = [None if g is None else np.ascontiguousarray(g, dtype=np.float64) for g in grads]
+    dp = ctypes.POINTER(ctypes.c_double)
+    P = (dp * n)(*[_dptr(p) for p in params])
+    G = (dp * n)(*[(_dptr(g) if g is not None else dp()) for g in g64])
+    M = (dp * n)(*[_dptr(m) for m in exp_avg])
+    V = (dp * n)(*[_dptr(v) for v in exp_avg_sq])
+    numel = np.array([p.size for p in params], dtype=np.int64)
+    rc = lib.oracle_adamw_step(n, P, G, M, V, numel.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), step, lr,
+                               beta1, beta2, eps, weight_decay)
+    if rc != 0:
+        raise ValueError("oracle_adamw_step rejected its arguments")

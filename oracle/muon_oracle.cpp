@@ -1,4 +1,5 @@
-// Plain fp64 reference of the Muon optimizer step: TEST INFRASTRUCTURE ONLY.
+// Plain fp64 reference of the Muon optimizer step (and of the AdamW step for the
+// parameters Muon leaves out): TEST INFRASTRUCTURE ONLY.
 //
 // Only the tests, the smoke check and the benchmark's CPU-baseline leg may
 // load this library. The product path (the CUDA library) never calls it and
@@ -17,6 +18,9 @@
 //     mean over dim 0, taken before the momentum buffer (section 4.2 order);
 //     section 2.2: the cubic iteration X = 1.5 X - 0.5 X X^T X; section 4.2:
 //     decoupled weight decay p *= (1 - lr wd) before the update.
+//   * "Muon meets Mamba" section 4.2 `_step_adamw` (and the moment equations of
+//     section 1.3): the AdamW step, with bias correction and decoupled decay,
+//     for the parameters that do not go to Muon.
 //   * "AdamW vs Muon" (adg.csdn.net), part 3 "scaling and update": RMS rescale
 //     by matrix shape, then times lr, then weight decay and subtraction; the
 //     quintic written as M_k = a M + b (M M^T) M + c (M M^T)^2 M; the
@@ -182,6 +186,40 @@ int oracle_muon_step(int count, double* const* params, const double* const* grad
     double* p = params[i];
     for (i64 e = 0; e < n_el; ++e) p[e] = p[e] * (1.0 - lr * weight_decay) - lr * s * O[e];
     if (O_out && O_out[i]) std::memcpy(O_out[i], O.data(), sizeof(double) * n_el);
+  }
+  return 0;
+}
+
+// One AdamW step over `count` tensors of numel[i] elements (the `_step_adamw` routine of
+// "Muon meets Mamba" section 4.2, for the parameters that do not go to Muon: embeddings, head,
+// norms, biases), in this order:
+//   p  <- p (1 - lr wd)                            (decoupled weight decay, first)
+//   m  <- beta1 m + (1 - beta1) g
+//   v  <- beta2 v + (1 - beta2) g^2
+//   p  <- p - (lr / (1 - beta1^t)) m / (sqrt(v) / sqrt(1 - beta2^t) + eps)
+// with t = step, the step count after this step (t >= 1). grads[i] == NULL skips tensor i.
+int oracle_adamw_step(int count, double* const* params, const double* const* grads,
+                      double* const* exp_avg, double* const* exp_avg_sq, const i64* numel, i64 step,
+                      double lr, double beta1, double beta2, double eps, double weight_decay) {
+  if (count < 0 || step < 1) return -1;
+  if (count > 0 && (!params || !grads || !exp_avg || !exp_avg_sq || !numel)) return -1;
+  const double bias_corr1 = 1.0 - std::pow(beta1, (double)step);
+  const double bias_corr2 = 1.0 - std::pow(beta2, (double)step);
+  const double step_size = lr / bias_corr1;
+  for (int i = 0; i < count; ++i) {
+    if (!grads[i]) continue;
+    if (numel[i] < 0 || !params[i] || !exp_avg[i] || !exp_avg_sq[i]) return -1;
+    double* p = params[i];
+    double* m = exp_avg[i];
+    double* v = exp_avg_sq[i];
+    const double* g = grads[i];
+    for (i64 e = 0; e < numel[i]; ++e) {
+      if (weight_decay != 0.0) p[e] = p[e] * (1.0 - lr * weight_decay);
+      m[e] = beta1 * m[e] + (1.0 - beta1) * g[e];
+      v[e] = beta2 * v[e] + (1.0 - beta2) * g[e] * g[e];
+      const double denom = std::sqrt(v[e]) / std::sqrt(bias_corr2) + eps;
+      p[e] = p[e] - step_size * m[e] / denom;
+    }
   }
   return 0;
 }

@@ -254,8 +254,50 @@ def pin_checkpoint_split(lib) -> None:
     assert np.array_equal(p_c, p_a) and np.array_equal(m_c, m_a)
 
 
+def _adamw(lib, p, g_list, lr, b1, b2, eps, wd, m=None, v=None, step0=0):
+    m = np.zeros_like(p) if m is None else m
+    v = np.zeros_like(p) if v is None else v
+    for t, g in enumerate(g_list, start=step0 + 1):
+        oracle.adamw_step([p], [g], [m], [v], step=t, lr=lr, beta1=b1, beta2=b2, eps=eps, weight_decay=wd,
+                          lib=lib)
+    return p, m, v
+
+
+def pin_adamw_golden(lib) -> None:
+    """AdamW against the hand-worked two-step example ("Muon meets Mamba" 4.2 `_step_adamw`)."""
+    g = read_golden("adamw_2step.txt")
+    p = g["p0"].copy(); m = np.zeros(2); v = np.zeros(2)
+    kw = dict(lr=float(g["lr"][0]), beta1=float(g["b1"][0]), beta2=float(g["b2"][0]), eps=0.0,
+              weight_decay=float(g["wd"][0]), lib=lib)
+    oracle.adamw_step([p], [g["g1"]], [m], [v], step=1, **kw)
+    assert np.max(np.abs(m - g["m1"])) < 1e-15 and np.max(np.abs(v - g["v1"])) < 1e-15
+    assert np.max(np.abs(p - g["p1"])) < 1e-15
+    oracle.adamw_step([p], [g["g2"]], [m], [v], step=2, **kw)
+    assert np.max(np.abs(m - g["m2"])) < 1e-15 and np.max(np.abs(v - g["v2"])) < 1e-15
+    assert np.max(np.abs(p - g["p2"])) < 1e-14
+    _, m, v = _adamw(lib, np.zeros(2), [g["g1"], np.array([0.0, 3.0])], lr=0.0, b1=0.9, b2=0.99, eps=1e-8, wd=0.0)
+    assert np.max(np.abs(m - g["bm2"])) < 1e-15 and np.max(np.abs(v - g["bv2"])) < 1e-15
+
+
+def pin_adamw_closed_forms(lib) -> None:
+    """With bias correction, a constant gradient g moves every weight by -lr g / (|g| + eps) at every
+    step (the corrected moments are g and g^2 exactly); the first step from zero state is the same;
+    a zero gradient leaves only the decoupled decay p (1 - lr wd)."""
+    r = rng(21)
+    g = r.standard_normal(40) * np.exp(r.uniform(-6, 2, 40))
+    p0 = r.standard_normal(40)
+    lr, eps = 1e-2, 1e-8
+    for t_total in (1, 7):
+        p, _, _ = _adamw(lib, p0.copy(), [g] * t_total, lr=lr, b1=0.9, b2=0.95, eps=eps, wd=0.0)
+        want = p0 - t_total * lr * g / (np.abs(g) + eps)
+        assert np.max(np.abs(p - want)) < 1e-12 * t_total, t_total
+    p, m, v = _adamw(lib, p0.copy(), [np.zeros(40)] * 3, lr=lr, b1=0.9, b2=0.95, eps=eps, wd=0.1)
+    assert np.max(np.abs(p - p0 * (1 - lr * 0.1) ** 3)) < 1e-15 and not m.any() and not v.any()
+
+
 ALL_PINS = [pin_spectral_map, pin_rank_one, pin_diagonal, pin_cubic_converges_to_polar, pin_quintic_band,
-            pin_invariances, pin_momentum_golden, pin_update_rule, pin_zero_center, pin_checkpoint_split]
+            pin_invariances, pin_momentum_golden, pin_update_rule, pin_zero_center, pin_checkpoint_split,
+            pin_adamw_golden, pin_adamw_closed_forms]
 
 
 def failing_pins(lib) -> List[str]:

@@ -30,6 +30,12 @@ MUTANTS = {
     "center_wrong_divisor": ("mean[j] /= (double)r;", "mean[j] /= (double)c;"),
     "center_after_momentum": ("if (zero_center) zero_center_rows(g.data(), r, c);", ""),
     "matmul_accumulate_index": ("c[j] += a * b[j];", "c[j] += a * b[(j + 1) % N];"),
+    "adamw_no_bias_corr1": ("const double step_size = lr / bias_corr1;", "const double step_size = lr;"),
+    "adamw_no_bias_corr2": ("std::sqrt(v[e]) / std::sqrt(bias_corr2) + eps", "std::sqrt(v[e]) + eps"),
+    "adamw_second_moment_not_squared": ("(1.0 - beta2) * g[e] * g[e]", "(1.0 - beta2) * g[e]"),
+    "adamw_decay_after_update": ("if (weight_decay != 0.0) p[e] = p[e] * (1.0 - lr * weight_decay);",
+                                 "if (weight_decay != 0.0) p[e] = p[e] * (1.0 - weight_decay);"),
+    "adamw_momentum_coeff": ("m[e] = beta1 * m[e] + (1.0 - beta1) * g[e];", "m[e] = beta1 * m[e] + g[e];"),
 }
 
 
