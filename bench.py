@@ -309,6 +309,8 @@ def run_ours(args, world, rank, local):
 
     if args.e2e:
         result["e2e"] = run_e2e(args, wl, ns, params, grads, mom, stream, world, device)
+    if args.adamw:
+        result["adamw"] = run_adamw(args, ns, stream, world, device, hbm_peak, peak_src)
     if args.cpu_baseline and rank == 0 and world == 1:
         result["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[args.workload], os.cpu_count() or 1)
     if rank == 0:
@@ -355,6 +357,50 @@ def run_e2e(args, wl, ns, params, grads, mom, stream, world, device):
                     "stays resident in HBM"}
 
 
+def run_adamw(args, ns, stream, world, device, hbm_peak, peak_src):
+    """AdamW step of the parameters the Muon step leaves out (Llama-8B token embedding and head,
+    65 RMSNorm scales: 1.05e9 elements), timed on its own: one launch per step, HBM-bound."""
+    import torch
+    awl = synth.ADAM_WORKLOADS["llama8b_adamw"]
+    ps = [awl.param_torch(i, device).to(torch.float32) for i in range(awl.count)]
+    gs = [awl.grad_torch(i, 1, device).to(torch.bfloat16) for i in range(awl.count)]
+    ms = [torch.zeros_like(p) for p in ps]
+    vs = [torch.zeros_like(p) for p in ps]
+    torch.cuda.synchronize()
+    kw = dict(lr=awl.lr, beta1=awl.beta1, beta2=awl.beta2, eps=awl.eps, weight_decay=awl.weight_decay,
+              stream=stream)
+    t = 0
+    for _ in range(args.warmup):
+        t += 1
+        ns.adamw_step(ps, gs, ms, vs, step=t, **kw)
+    ns.profile_read()
+    ns.profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, device)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        t += 1
+        ns.adamw_step(ps, gs, ms, vs, step=t, **kw)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    prof = ns.profile_read()
+    ns.profile_enable(False)
+    ms_step = reduce_max(ev0.elapsed_time(ev1), world, device) / args.steps
+    kernel_ms = prof["adamw"][1] / max(prof["adamw"][0], 1)
+    elements = awl.elements()
+    bytes_step = elements * (4 + 2 + 4 + 4 + 4 + 4 + 4)   # read p, g (bf16), m, v; write p, m, v
+    achieved = bytes_step / (kernel_ms * 1e-3) / 1e9
+    del ps, gs, ms, vs
+    torch.cuda.empty_cache()
+    return {"workload": awl.name, "elements": elements, "ms_per_step": ms_step,
+            "kernel_ms": kernel_ms, "launches_per_step": prof["adamw"][0] / args.steps,
+            "value": world * awl.count / (ms_step / 1e3), "unit": "tensors/s",
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved / hbm_peak, "traffic": None,
+                         "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                         "bytes_definition": "26 B per element: p, bf16 g, m, v read; p, m, v written"}}
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, world, rank):
     if rank != 0:
@@ -392,6 +438,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-adamw", dest="adamw", action="store_false",
+                    help="skip the AdamW measurement on the parameters Muon leaves out")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

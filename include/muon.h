@@ -165,6 +165,29 @@ MUON_API int muon_ns_orthogonalize_noalloc(const void* G, muon_dtype_t g_dtype, 
                                            const muon_coeffs_t* coeffs, float eps, int* status,
                                            muon_stream_t stream);
 
+/*
+ * One AdamW step over `count` tensors, for the parameters that do not go to Muon (embeddings,
+ * prediction head, norm scales, biases: "Muon meets Mamba" sections 2.1 and 4.3; "AdamW vs Muon"
+ * on which modules keep AdamW). Follows `_step_adamw` ("Muon meets Mamba" section 4.2):
+ *
+ *   p <- p (1 - lr wd)                                           decoupled decay, first
+ *   m <- beta1 m + (1 - beta1) g,   v <- beta2 v + (1 - beta2) g^2
+ *   p <- p - (lr / (1 - beta1^t)) m / (sqrt(v) / sqrt(1 - beta2^t) + eps)
+ *
+ *   params[i], exp_avg[i], exp_avg_sq[i]   device fp32, numel[i] elements each (any shape,
+ *                  contiguous); updated in place. Start the moments from zeros.
+ *   grads[i]       device, element type grad_dtype; NULL skips tensor i.
+ *   step           t, the step count after this step (1 for the first step); shared by all tensors.
+ *   lr, beta1, beta2, eps, weight_decay   0 <= beta < 1, eps >= 0, lr and wd finite
+ *                  (the pages' defaults: lr 1e-3, betas (0.9, 0.95), eps 1e-8).
+ * Arithmetic is fp32. One launch covers every tensor. Buffers of different tensors must not
+ * overlap. Returns MUON_OK or a negative error code.
+ */
+MUON_API int muon_adamw_step(int count, float* const* params, const void* const* grads,
+                             muon_dtype_t grad_dtype, float* const* exp_avg, float* const* exp_avg_sq,
+                             const int64_t* numel, int64_t step, float lr, float beta1, float beta2,
+                             float eps, float weight_decay, muon_stream_t stream);
+
 /* Message describing the last error returned on the calling thread ("" if none). The pointer
  * stays valid until the next call on that thread. */
 MUON_API const char* muon_last_error(void);
@@ -185,7 +208,8 @@ enum {
   MUON_KC_NORM = 2,     /* per-matrix 1 / (||u|| + eps)                                 */
   MUON_KC_GEMM = 3,     /* Newton-Schulz matrix products (all three phases)             */
   MUON_KC_EPILOGUE = 4, /* decay and parameter update, or the output conversion         */
-  MUON_KC_COUNT = 5
+  MUON_KC_ADAMW = 5,    /* AdamW step (muon_adamw_step)                                 */
+  MUON_KC_COUNT = 6
 };
 
 /* Turns per-launch timing on (nonzero) or off. While on, every kernel launch is bracketed by

@@ -21,16 +21,16 @@ PREC_BF16, PREC_FP32 = 0, 1
 RMS_ONE, RMS_SQRT_MAX1_ROWS_OVER_COLS = 0, 1
 OK, WARN_NONFINITE = 0, 1
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = -1, -2, -3, -4, -5
-KC_CENTER, KC_PROLOGUE, KC_NORM, KC_GEMM, KC_EPILOGUE, KC_COUNT = 0, 1, 2, 3, 4, 5
-KC_NAMES = ["center", "prologue", "norm", "gemm", "epilogue"]
+KC_CENTER, KC_PROLOGUE, KC_NORM, KC_GEMM, KC_EPILOGUE, KC_ADAMW, KC_COUNT = 0, 1, 2, 3, 4, 5, 6
+KC_NAMES = ["center", "prologue", "norm", "gemm", "epilogue", "adamw"]
 MAX_NS_STEPS = 64
 
 QUINTIC = (3.4445, -4.7750, 2.0315)
 CUBIC = (1.5, -0.5, 0.0)
 
-EXPORTS = ["muon_ns_orthogonalize", "muon_step", "muon_last_error", "muon_check_status",
-           "muon_release_workspace", "muon_profile_enable", "muon_profile_read", "muon_launch_count",
-           "muon_version"]
+EXPORTS = ["muon_ns_orthogonalize", "muon_step", "muon_adamw_step", "muon_last_error",
+           "muon_check_status", "muon_release_workspace", "muon_profile_enable", "muon_profile_read",
+           "muon_launch_count", "muon_version"]
 
 
 class MuonError(RuntimeError):
@@ -58,6 +58,10 @@ def _load() -> ctypes.CDLL:
     lib.muon_step.argtypes = [ctypes.c_int, vpp, vpp, ctypes.c_int, vpp, i64p, i64p, ctypes.c_float,
                               ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int,
                               ctypes.POINTER(Coeffs), ctypes.c_int, ctypes.c_float, ctypes.c_int, vp]
+    lib.muon_adamw_step.restype = ctypes.c_int
+    lib.muon_adamw_step.argtypes = [ctypes.c_int, vpp, vpp, ctypes.c_int, vpp, vpp, i64p, ctypes.c_int64,
+                                    ctypes.c_float, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                    ctypes.c_float, vp]
     lib.muon_last_error.restype = ctypes.c_char_p
     lib.muon_last_error.argtypes = []
     lib.muon_check_status.restype = ctypes.c_int
@@ -169,6 +173,35 @@ def muon_step(params: List, grads: List, momentum: List, lr: float = 0.02, mu: f
                          ctypes.cast(M, ctypes.POINTER(ctypes.c_void_p)), rows, cols, lr, mu,
                          int(nesterov), weight_decay, int(rms_scale), steps, co, int(zero_center), eps,
                          _prec_code(prec), _stream_handle(stream)))
+
+
+def adamw_step(params: List, grads: List, exp_avg: List, exp_avg_sq: List, step: int, lr: float = 1e-3,
+               beta1: float = 0.9, beta2: float = 0.95, eps: float = 1e-8, weight_decay: float = 0.0,
+               stream=None) -> None:
+    """One AdamW step over lists of contiguous CUDA tensors of any shape (params and moments fp32;
+    grads bf16 or fp32, all of one dtype; a None grad skips its tensor). `step` is the step count
+    after this step (1 for the first)."""
+    n = len(params)
+    if not (len(grads) == len(exp_avg) == len(exp_avg_sq) == n):
+        raise ValueError("params, grads, exp_avg and exp_avg_sq must have the same length")
+    g_dtype = None
+    for g in grads:
+        if g is not None:
+            code = _dtype_code(g)
+            if g_dtype is not None and code != g_dtype:
+                raise TypeError("all gradients must share one dtype")
+            g_dtype = code
+    if g_dtype is None:
+        return
+    VP = ctypes.c_void_p * max(1, n)
+    cast = lambda a: ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
+    P = VP(*[p.data_ptr() for p in params])
+    G = VP(*[(g.data_ptr() if g is not None else None) for g in grads])
+    M = VP(*[m.data_ptr() for m in exp_avg])
+    V = VP(*[v.data_ptr() for v in exp_avg_sq])
+    N = (ctypes.c_int64 * max(1, n))(*[p.numel() for p in params])
+    _check(lib.muon_adamw_step(n, cast(P), cast(G), g_dtype, cast(M), cast(V), N, step, lr, beta1, beta2,
+                               eps, weight_decay, _stream_handle(stream)))
 
 
 def check_status(stream=None) -> int:

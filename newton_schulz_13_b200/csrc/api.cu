@@ -159,7 +159,25 @@ struct Plan {
   }
 };
 
+// Per-device table of an AdamW call: one AdamTensor per tensor, re-uploaded (from pinned staging)
+// only when the pointers change.
+struct AdamPlan {
+  std::vector<int64_t> numel;
+  AdamTensor* d_tab = nullptr;
+  AdamTensor* h_pinned = nullptr;
+  cudaEvent_t done = nullptr;
+  std::vector<AdamTensor> last;
+  bool uploaded = false;
+  int64_t n_chunks = 0;
+  ~AdamPlan() {
+    if (done) cudaEventDestroy(done);
+    if (h_pinned) cudaFreeHost(h_pinned);
+    if (d_tab) cudaFree(d_tab);
+  }
+};
+
 struct DeviceState {
+  std::unique_ptr<AdamPlan> adam;
   std::unique_ptr<Plan> plan;
   int* d_status = nullptr;  // [0] flags, [1] non-finite count
   int sms = 0;
@@ -725,6 +743,7 @@ int muon_release_workspace(void) {
   if (it == g_dev.end()) return MUON_OK;
   cudaDeviceSynchronize();
   it->second.plan.reset();
+  it->second.adam.reset();
   return MUON_OK;
 }
 
@@ -826,6 +845,94 @@ int muon_step(int count, float* const* params, const void* const* grads, muon_dt
                          ew_grid, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
+  return MUON_OK;
+}
+
+int muon_adamw_step(int count, float* const* params, const void* const* grads, muon_dtype_t grad_dtype,
+                    float* const* exp_avg, float* const* exp_avg_sq, const int64_t* numel, int64_t step,
+                    float lr, float beta1, float beta2, float eps, float weight_decay, muon_stream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  t_err.clear();
+  if (count < 0) return fail(MUON_ERR_INVALID_ARG, "count must be >= 0");
+  if (count > 0 && (!params || !grads || !exp_avg || !exp_avg_sq || !numel))
+    return fail(MUON_ERR_INVALID_ARG, "params, grads, exp_avg, exp_avg_sq and numel must not be NULL");
+  if (grad_dtype != MUON_BF16 && grad_dtype != MUON_FP32) return fail(MUON_ERR_INVALID_ARG, "grad_dtype");
+  if (step < 1) return fail(MUON_ERR_INVALID_ARG, "step must be >= 1 (the step count after this step)");
+  if (!finite_f(lr) || !finite_f(weight_decay)) return fail(MUON_ERR_INVALID_ARG, "lr and weight_decay must be finite");
+  if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f))
+    return fail(MUON_ERR_INVALID_ARG, "beta1 and beta2 must be in [0, 1)");
+  if (!(eps >= 0.0f) || !finite_f(eps)) return fail(MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  std::vector<int> idx;
+  Ranges written;
+  for (int i = 0; i < count; ++i) {
+    if (!grads[i] || numel[i] == 0) continue;
+    if (numel[i] < 0 || numel[i] > (int64_t(1) << 36)) return fail(MUON_ERR_INVALID_ARG, "numel out of range");
+    if (!params[i] || !exp_avg[i] || !exp_avg_sq[i])
+      return fail(MUON_ERR_INVALID_ARG, "params[i], exp_avg[i] and exp_avg_sq[i] must not be NULL");
+    const size_t bytes = (size_t)numel[i] * 4;
+    written.add(params[i], bytes);
+    written.add(exp_avg[i], bytes);
+    written.add(exp_avg_sq[i], bytes);
+    idx.push_back(i);
+  }
+  if (written.overlap()) return fail(MUON_ERR_INVALID_ARG, "params/exp_avg/exp_avg_sq buffers overlap");
+  if (idx.empty()) return MUON_OK;
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != MUON_OK) return rc;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int n = (int)idx.size();
+  std::vector<int64_t> nel(n);
+  for (int j = 0; j < n; ++j) nel[j] = numel[idx[j]];
+  if (!ds->adam || ds->adam->numel != nel) {
+    ds->adam.reset();
+    std::unique_ptr<AdamPlan> A(new AdamPlan());
+    A->numel = nel;
+    MUON_CUDA(cudaMalloc(&A->d_tab, (size_t)n * sizeof(AdamTensor)));
+    MUON_CUDA(cudaMallocHost(&A->h_pinned, (size_t)n * sizeof(AdamTensor)));
+    MUON_CUDA(cudaEventCreateWithFlags(&A->done, cudaEventDisableTiming));
+    ds->adam = std::move(A);
+  }
+  AdamPlan& A = *ds->adam;
+  std::vector<AdamTensor> tab(n);
+  int64_t chunks = 0;
+  for (int j = 0; j < n; ++j) {
+    const int i = idx[j];
+    AdamTensor& t = tab[j];
+    std::memset(&t, 0, sizeof(t));
+    t.p = params[i];
+    t.g = grads[i];
+    t.m = exp_avg[i];
+    t.v = exp_avg_sq[i];
+    t.numel = numel[i];
+    t.chunk_begin = chunks;
+    chunks += ceil_div(numel[i], kChunk);
+    t.vec = ((uintptr_t)params[i] % 16 == 0 && (uintptr_t)grads[i] % 16 == 0 &&
+             (uintptr_t)exp_avg[i] % 16 == 0 && (uintptr_t)exp_avg_sq[i] % 16 == 0) ? 1 : 0;
+  }
+  A.n_chunks = chunks;
+  if (!A.uploaded || std::memcmp(tab.data(), A.last.data(), n * sizeof(AdamTensor)) != 0) {
+    MUON_CUDA(cudaEventSynchronize(A.done));
+    std::memcpy(A.h_pinned, tab.data(), n * sizeof(AdamTensor));
+    MUON_CUDA(cudaMemcpyAsync(A.d_tab, A.h_pinned, n * sizeof(AdamTensor), cudaMemcpyHostToDevice, s));
+    MUON_CUDA(cudaEventRecord(A.done, s));
+    A.last = tab;
+    A.uploaded = true;
+  }
+  const double bc1 = 1.0 - std::pow((double)beta1, (double)step);
+  const double bc2 = 1.0 - std::pow((double)beta2, (double)step);
+  AdamScalars sc;
+  sc.decay = 1.0f - lr * weight_decay;
+  sc.beta1 = beta1;
+  sc.beta2 = beta2;
+  sc.step_size = (float)((double)lr / bc1);
+  sc.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(bc2));
+  sc.eps = eps;
+  const int g_bf16 = grad_dtype == MUON_BF16;
+  cudaError_t e = timed_launch(MUON_KC_ADAMW, s, 0, 0, [&] {
+    return launch_adamw(A.d_tab, n, A.n_chunks, g_bf16, sc, ds->sms * 4, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "adamw launch");
   return MUON_OK;
 }
 

@@ -341,11 +341,85 @@ __global__ void __launch_bounds__(kEwThreads) output_kernel(const MatInfo* __res
   }
 }
 
+// ---------------------------------------------------------------- AdamW
+// The AdamW step of the parameters Muon leaves out ("Muon meets Mamba" 4.2 `_step_adamw`):
+// decoupled decay first, then bias-corrected first and second moments. 4 fp32 arrays plus the
+// gradient per element: 26 B (bf16 gradient) or 28 B (fp32) of HBM traffic.
+__device__ __forceinline__ int find_tensor(const AdamTensor* ts, int n, int64_t chunk) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ts[mid].chunk_begin <= chunk) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void adam_elem(float& p, float& m, float& v, float g, const AdamScalars& sc) {
+  p = p * sc.decay;
+  m = sc.beta1 * m + (1.0f - sc.beta1) * g;
+  v = sc.beta2 * v + (1.0f - sc.beta2) * g * g;
+  p = p - sc.step_size * m / (sqrtf(v) * sc.inv_sqrt_bc2 + sc.eps);
+}
+
+template <bool G_BF16>
+__global__ void __launch_bounds__(kEwThreads, 4) adamw_kernel(const AdamTensor* __restrict__ ts, int n,
+                                                              int64_t nchunks, AdamScalars sc) {
+  for (int64_t chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
+    const int j = find_tensor(ts, n, chunk);
+    const AdamTensor t = ts[j];
+    const int64_t e0 = (chunk - t.chunk_begin) * kChunk;
+    const int64_t e1 = min(t.numel, e0 + kChunk);
+    if (t.vec) {
+      const int64_t nvec = (e1 - e0) / 8;   // whole groups of 8; the rest below
+      constexpr int kBatch = 1;             // 4 arrays x 8 values already fill the register budget
+      for (int64_t q0 = threadIdx.x; q0 < nvec; q0 += (int64_t)kBatch * blockDim.x) {
+        float g[kBatch][8], p[kBatch][8], m[kBatch][8], v[kBatch][8];
+        bool ok[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          const int64_t q = q0 + (int64_t)b * blockDim.x;
+          ok[b] = q < nvec;
+          if (ok[b]) {
+            const int64_t e = e0 + 8 * q;
+            load8<G_BF16>(t.g, e, g[b]);
+            load8<false>(t.p, e, p[b]);
+            load8<false>(t.m, e, m[b]);
+            load8<false>(t.v, e, v[b]);
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+          if (!ok[b]) continue;
+          const int64_t e = e0 + 8 * (q0 + (int64_t)b * blockDim.x);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) adam_elem(p[b][i], m[b][i], v[b][i], g[b][i], sc);
+          store8<false>(t.p, e, p[b]);
+          store8<false>(t.m, e, m[b]);
+          store8<false>(t.v, e, v[b]);
+        }
+      }
+      for (int64_t e = e0 + 8 * nvec + threadIdx.x; e < e1; e += blockDim.x)
+        adam_elem(t.p[e], t.m[e], t.v[e], load1<G_BF16>(t.g, e), sc);
+    } else {
+      for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x)
+        adam_elem(t.p[e], t.m[e], t.v[e], load1<G_BF16>(t.g, e), sc);
+    }
+  }
+}
+
 int grid_for(int64_t items, int cap) {
   return (int)(items < (int64_t)cap ? (items < 1 ? 1 : items) : cap);
 }
 
 }  // namespace
+
+cudaError_t launch_adamw(const AdamTensor* ts, int n, int64_t chunks, int g_bf16, AdamScalars sc,
+                         int grid, cudaStream_t s) {
+  grid = grid_for(chunks, grid);
+  if (g_bf16) adamw_kernel<true><<<grid, kEwThreads, 0, s>>>(ts, n, chunks, sc);
+  else adamw_kernel<false><<<grid, kEwThreads, 0, s>>>(ts, n, chunks, sc);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_colsum(const MatInfo* mats, int nmats, int64_t items, int g_bf16, cudaStream_t s) {
   const int grid = grid_for(items, 148 * 16);

@@ -39,6 +39,24 @@ struct MatInfo {
   int vec;             // 1: 16-byte vector path is legal (cols % 8 == 0, aligned pointers)
 };
 
+// One tensor of an AdamW call (any shape, flattened).
+struct AdamTensor {
+  float* p;
+  const void* g;
+  float* m;
+  float* v;
+  int64_t numel;
+  int64_t chunk_begin;
+  int vec;             // 1: 16-byte vector path is legal (all four pointers 16-byte aligned)
+  int pad;
+};
+
+// Scalars of one AdamW step: p <- p decay; m <- b1 m + (1-b1) g; v <- b2 v + (1-b2) g^2;
+// p <- p - step_size m / (sqrt(v) inv_sqrt_bc2 + eps).
+struct AdamScalars {
+  float decay, beta1, beta2, step_size, inv_sqrt_bc2, eps;
+};
+
 // One problem of a grouped tensor-core launch:
 //   D = s_acc * (opA . opB^T) + s_c * C,   D: M x N, contraction over K,
 // where opA(i, k) and opB(j, k) are read through TMA from bf16 matrices either K-major
@@ -101,6 +119,8 @@ cudaError_t launch_update(const MatInfo* mats, int nmats, int64_t chunks, int x_
                           float decay, int scale_by_alpha, int grid, cudaStream_t s);
 cudaError_t launch_output(const MatInfo* mats, int nmats, int64_t chunks, int x_bf16, int out_bf16,
                           int scale_by_alpha, int grid, cudaStream_t s);
+cudaError_t launch_adamw(const AdamTensor* ts, int n, int64_t chunks, int g_bf16, AdamScalars sc,
+                         int grid, cudaStream_t s);
 cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                            EpiScalars ep, int* status, int grid, cudaStream_t s);
 cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,

@@ -262,6 +262,65 @@ WORKLOADS["llama8b_layer"] = Workload(**{**WORKLOADS["llama8b"].__dict__, "name"
                                          "description": "one layer of the Llama-8B hidden-weight set",
                                          "shapes": WORKLOADS["llama8b"].shapes[:7]})
 
+# ----------------------------------------------------------------------------
+# AdamW workloads: the parameters that do not go to Muon (embeddings, head, norms, biases)
+# ----------------------------------------------------------------------------
+
+@dataclass
+class AdamWorkload:
+    name: str
+    description: str
+    sizes: List[int]                # numel of each tensor
+    grad_dtype: str
+    grad_std: float
+    param_std: float
+    seed: int
+    lr: float
+    beta1: float
+    beta2: float
+    eps: float
+    weight_decay: float
+    n_steps: int
+
+    @property
+    def count(self) -> int:
+        return len(self.sizes)
+
+    def elements(self) -> int:
+        return sum(self.sizes)
+
+    def grad(self, i: int, step: int) -> np.ndarray:
+        return standard_normal(matrix_key(self.seed, i, KIND_GRAD, step), self.sizes[i]) * self.grad_std
+
+    def param(self, i: int) -> np.ndarray:
+        return standard_normal(matrix_key(self.seed, i, KIND_PARAM, 0), self.sizes[i]) * self.param_std
+
+    def grad_torch(self, i: int, step: int, device):
+        return standard_normal_torch(matrix_key(self.seed, i, KIND_GRAD, step), self.sizes[i], device) * self.grad_std
+
+    def param_torch(self, i: int, device):
+        return standard_normal_torch(matrix_key(self.seed, i, KIND_PARAM, 0), self.sizes[i], device) * self.param_std
+
+
+_GPT2_SMALL_ADAM = ([50257 * 768, 1024 * 768]                             # token and position embeddings
+                    + [768, 768, 2304, 768, 768, 768, 3072, 768] * 12     # per layer: ln1 w/b, qkv b, proj b,
+                    + [768, 768])                                          # ln2 w/b, fc b, fc-proj b; final ln
+_LLAMA8B_ADAM = [128256 * 4096, 128256 * 4096] + [4096] * 65               # embedding, head, 2 norms x 32 + final
+
+ADAM_WORKLOADS = {
+    "gpt2_small_adamw": AdamWorkload(
+        name="gpt2_small_adamw",
+        description="GPT-2-small parameters outside Muon: embeddings, layer-norm scales and shifts, biases",
+        sizes=_GPT2_SMALL_ADAM, grad_dtype="bf16", grad_std=1e-3, param_std=0.02, seed=13, lr=1e-3,
+        beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.01, n_steps=3),
+    "llama8b_adamw": AdamWorkload(
+        name="llama8b_adamw",
+        description="Llama-8B parameters outside Muon: token embedding and prediction head (128256 x 4096), "
+                    "65 RMSNorm scales of 4096",
+        sizes=_LLAMA8B_ADAM, grad_dtype="bf16", grad_std=1.0, param_std=0.02, seed=15, lr=1e-3,
+        beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, n_steps=1),
+}
+
 # The eight-plus-two coefficient schedule (eight quintic iterations, then two
 # with (2, -1.5, 0.5)), exercised on the GPT-2-small shapes.
 HYBRID = [(3.445, -4.7750, 2.0315)] * 8 + [(2.0, -1.5, 0.5)] * 2

@@ -21,7 +21,7 @@ def test_header_declares_the_entry_points():
     names = declared_symbols()
     for n in ("muon_ns_orthogonalize", "muon_step", "muon_last_error", "muon_check_status",
               "muon_release_workspace", "muon_profile_enable", "muon_profile_read", "muon_launch_count",
-              "muon_version", "muon_ns_orthogonalize_noalloc"):
+              "muon_version", "muon_ns_orthogonalize_noalloc", "muon_adamw_step"):
         assert n in names
 
 
@@ -132,3 +132,40 @@ def test_profile_read_without_launches():
     rec = ns.profile_read()
     assert set(rec) == set(ns.KC_NAMES) and all(v[0] == 0 for v in rec.values())
     assert ns.version() >= 100
+
+
+def _adam(ns, count=1, params=None, grads=None, m=None, v=None, numel=None, step=1, lr=1e-3, b1=0.9,
+          b2=0.95, eps=1e-8, wd=0.0, gdt=0):
+    VP = ctypes.c_void_p * max(count, 1)
+    cast = lambda a: ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
+    P = VP(*(params or [0x100000 * (i + 1) for i in range(count)]))
+    G = VP(*(grads or [0x90000000 + 0x100000 * i for i in range(count)]))
+    M = VP(*(m or [0x50000000 + 0x100000 * i for i in range(count)]))
+    V = VP(*(v or [0x70000000 + 0x100000 * i for i in range(count)]))
+    N = (ctypes.c_int64 * max(count, 1))(*(numel or [16] * count))
+    return ns.lib.muon_adamw_step(count, cast(P), cast(G), gdt, cast(M), cast(V), N, step, lr, b1, b2, eps, wd, None)
+
+
+@pytest.mark.parametrize("kw,needle", [
+    (dict(count=-1), "count"),
+    (dict(step=0), "step"),
+    (dict(b1=1.0), "beta"),
+    (dict(b2=-0.5), "beta"),
+    (dict(eps=-1e-8), "eps"),
+    (dict(lr=float("nan")), "lr"),
+    (dict(gdt=5), "grad_dtype"),
+    (dict(numel=[-3]), "numel"),
+    (dict(params=[0x1000], m=[0x1010]), "overlap"),
+    (dict(count=2, params=[0x1000, 0x9000], v=[0x20000, 0x9020]), "overlap"),
+])
+def test_adamw_rejects_bad_arguments(kw, needle):
+    import newton_schulz_13_b200 as ns
+    assert _adam(ns, **kw) == ns.ERR_INVALID_ARG
+    assert needle in ns.last_error()
+
+
+@pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="checks the no-device path")
+def test_adamw_no_device_fails_loudly():
+    import newton_schulz_13_b200 as ns
+    assert _adam(ns) == ns.ERR_UNSUPPORTED
+    assert _adam(ns, numel=[0]) == ns.OK   # nothing to do: no device needed
