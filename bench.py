@@ -212,21 +212,32 @@ def run_ours(args, world, rank, local):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
     wl = synth.WORKLOADS[args.workload]
-    # every rank owns an independent weight set of the same shapes (weak scaling)
-    wl = synth.Workload(**{**wl.__dict__, "seed": wl.seed + 1000 * rank})
+    if not args.sharded:
+        # every rank owns an independent weight set of the same shapes (weak scaling)
+        wl = synth.Workload(**{**wl.__dict__, "seed": wl.seed + 1000 * rank})
+        owner = [rank] * wl.count
+    else:
+        # one weight set replicated on every rank; each rank updates its share of the matrices
+        # and the updated parameters are all-gathered (strong scaling)
+        from newton_schulz_13_b200 import sharded
+        owner = sharded.partition(wl.shapes, world)
     gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
     params, grads, mom = [], [], []
     for j in range(wl.count):
         params.append(wl.param_torch(j, device).to(torch.float32))
         grads.append(wl.grad_torch(j, 0, device).to(gdt))
-        mom.append(torch.zeros(wl.shapes[j], dtype=torch.float32, device=device))
+        mom.append(torch.zeros(wl.shapes[j], dtype=torch.float32, device=device) if owner[j] == rank else None)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream(device)
+    hp = dict(lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov, weight_decay=wl.weight_decay, rms_scale=wl.rms_scale,
+              steps=len(wl.coeffs), coeffs=wl.coeffs, zero_center=wl.zero_center, eps=wl.eps, prec="bf16",
+              stream=stream)
 
     def step():
-        ns.muon_step(params, grads, mom, lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov,
-                     weight_decay=wl.weight_decay, rms_scale=wl.rms_scale, steps=len(wl.coeffs),
-                     coeffs=wl.coeffs, zero_center=wl.zero_center, eps=wl.eps, prec="bf16", stream=stream)
+        if args.sharded:
+            sharded.sharded_muon_step(params, grads, mom, **hp)
+        else:
+            ns.muon_step(params, grads, mom, **hp)
 
     for _ in range(args.warmup):
         step()
@@ -253,7 +264,7 @@ def run_ours(args, world, rank, local):
     ns.profile_enable(False)
     status = max(status, ns.check_status())
     ms_step = ms_total / args.steps
-    value = world * wl.count / (ms_step / 1e3)
+    value = (1 if args.sharded else world) * wl.count / (ms_step / 1e3)
 
     peaks, peak_src = load_peaks()
     g_launch, g_ms, g_fl, g_ex = prof["gemm"]
@@ -274,7 +285,8 @@ def run_ours(args, world, rank, local):
 
     result = {
         "metric": METRIC, "value": value, "unit": "matrices/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if args.sharded else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "matrices_per_gpu": wl.count, "elements_per_gpu": elements,
                    "grad_dtype": wl.grad_dtype, "param_dtype": "fp32", "momentum_dtype": "fp32",
@@ -282,7 +294,9 @@ def run_ours(args, world, rank, local):
                    "weight_decay": wl.weight_decay, "rms_scale": "sqrt(max(1, rows/cols))",
                    "l2": "no flush: inputs (params+grads+momentum, %.0f GB per GPU) are larger than the "
                          "126 MB L2" % (elements * (4 + 4 + 2 * gbytes) / 1e9),
-                   "parallelism": "independent weight set per GPU (weak scaling, no collective)"},
+                   "parallelism": ("one weight set split across GPUs by Newton-Schulz FLOPs, updated parameters "
+                                   "all-gathered (strong scaling)") if args.sharded else
+                                  "independent weight set per GPU (weak scaling, no collective)"},
         "ns_tflops": achieved,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
@@ -308,7 +322,7 @@ def run_ours(args, world, rank, local):
     }
 
     if args.e2e:
-        result["e2e"] = run_e2e(args, wl, ns, params, grads, mom, stream, world, device)
+        result["e2e"] = run_e2e(args, wl, step, params, grads, stream, world, device)
     if args.adamw:
         result["adamw"] = run_adamw(args, ns, stream, world, device, hbm_peak, peak_src)
     if args.cpu_baseline and rank == 0 and world == 1:
@@ -320,7 +334,7 @@ def run_ours(args, world, rank, local):
         dist.destroy_process_group()
 
 
-def run_e2e(args, wl, ns, params, grads, mom, stream, world, device):
+def run_e2e(args, wl, step, params, grads, stream, world, device):
     """Same step through the public API with host buffers: every step copies the gradients from
     pinned host memory to the device and the updated parameters back, inside the timed region."""
     import torch
@@ -334,11 +348,9 @@ def run_e2e(args, wl, ns, params, grads, mom, stream, world, device):
     def e2e_step():
         for g, hg in zip(grads, h_grads):
             g.copy_(hg, non_blocking=True)
-        ns.muon_step(params, grads, mom, lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov,
-                     weight_decay=wl.weight_decay, rms_scale=wl.rms_scale, steps=len(wl.coeffs),
-                     coeffs=wl.coeffs, zero_center=wl.zero_center, eps=wl.eps, prec="bf16", stream=stream)
-        for hp, p in zip(h_params, params):
-            hp.copy_(p, non_blocking=True)
+        step()
+        for hp_, p in zip(h_params, params):
+            hp_.copy_(p, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -351,7 +363,8 @@ def run_e2e(args, wl, ns, params, grads, mom, stream, world, device):
     ev1.record(stream)
     torch.cuda.synchronize()
     ms = reduce_max(ev0.elapsed_time(ev1), world, device) / steps
-    return {"value": world * wl.count / (ms / 1e3), "unit": "matrices/s", "h2d_bytes_per_step": bi,
+    return {"value": (1 if args.sharded else world) * wl.count / (ms / 1e3), "unit": "matrices/s",
+            "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "ms_per_step": ms, "steps": steps,
             "note": "grads H2D from pinned host memory and updated fp32 params D2H every step; momentum "
                     "stays resident in HBM"}
@@ -438,6 +451,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--sharded", action="store_true",
+                    help="split one weight set across the GPUs and all-gather the updated parameters "
+                         "(strong scaling) instead of one independent weight set per GPU (weak scaling)")
     ap.add_argument("--no-adamw", dest="adamw", action="store_false",
                     help="skip the AdamW measurement on the parameters Muon leaves out")
     args = ap.parse_args(argv)
