@@ -371,10 +371,11 @@ def run_e2e(args, wl, step, params, grads, stream, world, device):
 
 
 def run_adamw(args, ns, stream, world, device, hbm_peak, peak_src):
-    """AdamW step of the parameters the Muon step leaves out (Llama-8B token embedding and head,
-    65 RMSNorm scales: 1.05e9 elements), timed on its own: one launch per step, HBM-bound."""
+    """AdamW step of the parameters the Muon step leaves out (by default the Llama-8B token
+    embedding and head and 65 RMSNorm scales: 1.05e9 elements), timed on its own: one launch per
+    step, HBM-bound."""
     import torch
-    awl = synth.ADAM_WORKLOADS["llama8b_adamw"]
+    awl = synth.ADAM_WORKLOADS[args.adamw_workload]
     ps = [awl.param_torch(i, device).to(torch.float32) for i in range(awl.count)]
     gs = [awl.grad_torch(i, 1, device).to(torch.bfloat16) for i in range(awl.count)]
     ms = [torch.zeros_like(p) for p in ps]
@@ -454,6 +455,7 @@ def main(argv=None):
     ap.add_argument("--sharded", action="store_true",
                     help="split one weight set across the GPUs and all-gather the updated parameters "
                          "(strong scaling) instead of one independent weight set per GPU (weak scaling)")
+    ap.add_argument("--adamw-workload", choices=sorted(synth.ADAM_WORKLOADS), default="llama8b_adamw")
     ap.add_argument("--no-adamw", dest="adamw", action="store_false",
                     help="skip the AdamW measurement on the parameters Muon leaves out")
     args = ap.parse_args(argv)

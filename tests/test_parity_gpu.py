@@ -66,6 +66,21 @@ def test_ns_orthogonalize_fp32(shape, sched):
     assert rel(host64(X), want) <= TOL_O_FP32, rel(host64(X), want)
 
 
+@pytest.mark.parametrize("shape", [(1 << 20, 16), (16, 1 << 20), (2, 1 << 20)], ids=lambda s: f"{s[0]}x{s[1]}")
+@pytest.mark.parametrize("sched", ["quintic5", "cubic5"], ids=str)
+def test_ns_largest_single_dimension(shape, sched):
+    """The largest row or column count the C ABI accepts (2^20), on thin matrices the oracle still
+    finishes in a second: Gram contractions over a million-long K, 4096 row tiles of the update."""
+    import newton_schulz_13_b200 as ns
+    co = SCHEDULES[sched]
+    G = synth.round_to(_gen(shape, 17), "bf16")
+    X = ns.ns_orthogonalize(to_dev(G, torch.bfloat16), steps=len(co), coeffs=co, eps=1e-7, prec="bf16",
+                            out_dtype=torch.float32)
+    assert ns.check_status() == ns.OK
+    want = oracle.newton_schulz(G, co, eps=1e-7)
+    assert rel(host64(X), want) <= TOL_O_BF16, rel(host64(X), want)
+
+
 @pytest.mark.parametrize("shape", [(96, 200), (200, 96), (64, 64)], ids=lambda s: f"{s[0]}x{s[1]}")
 def test_ns_zero_center(shape):
     import newton_schulz_13_b200 as ns
