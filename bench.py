@@ -316,6 +316,10 @@ def run_ours(args, world, rank, local):
                                                      ", bf16 O read + p read + p write (epilogue)"),
                                  "ms_per_step": ew_ms / args.steps},
         "kernels_ms_per_step": {k: v[1] / args.steps for k, v in prof.items()},
+        "ns_phases": {ph: {"ms_per_step": prof[k][1] / args.steps,
+                           "nominal_tflops": prof[k][2] / (prof[k][1] * 1e-3) / 1e12 if prof[k][1] else None,
+                           "executed_tflops": prof[k][3] / (prof[k][1] * 1e-3) / 1e12 if prof[k][1] else None}
+                      for ph, k in (("gram", "gemm_gram"), ("poly", "gemm_poly"), ("update", "gemm_update"))},
         "gpu_launches": launches,
         "clocks": clk.summary(),
         "status": status,

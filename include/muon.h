@@ -209,7 +209,12 @@ enum {
   MUON_KC_GEMM = 3,     /* Newton-Schulz matrix products (all three phases)             */
   MUON_KC_EPILOGUE = 4, /* decay and parameter update, or the output conversion         */
   MUON_KC_ADAMW = 5,    /* AdamW step (muon_adamw_step)                                 */
-  MUON_KC_COUNT = 6
+  /* breakdown of MUON_KC_GEMM by phase: every Newton-Schulz launch is counted both in
+   * MUON_KC_GEMM and in the class of its phase */
+  MUON_KC_GEMM_GRAM = 6,   /* A = X X^T                                                 */
+  MUON_KC_GEMM_POLY = 7,   /* B = c A A + b A (+ a I)                                   */
+  MUON_KC_GEMM_UPDATE = 8, /* X' = B X (last one may carry the fused parameter update)  */
+  MUON_KC_COUNT = 9
 };
 
 /* Turns per-launch timing on (nonzero) or off. While on, every kernel launch is bracketed by

@@ -21,8 +21,9 @@ PREC_BF16, PREC_FP32 = 0, 1
 RMS_ONE, RMS_SQRT_MAX1_ROWS_OVER_COLS = 0, 1
 OK, WARN_NONFINITE = 0, 1
 ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = -1, -2, -3, -4, -5
-KC_CENTER, KC_PROLOGUE, KC_NORM, KC_GEMM, KC_EPILOGUE, KC_ADAMW, KC_COUNT = 0, 1, 2, 3, 4, 5, 6
-KC_NAMES = ["center", "prologue", "norm", "gemm", "epilogue", "adamw"]
+KC_CENTER, KC_PROLOGUE, KC_NORM, KC_GEMM, KC_EPILOGUE, KC_ADAMW = 0, 1, 2, 3, 4, 5
+KC_GEMM_GRAM, KC_GEMM_POLY, KC_GEMM_UPDATE, KC_COUNT = 6, 7, 8, 9
+KC_NAMES = ["center", "prologue", "norm", "gemm", "epilogue", "adamw", "gemm_gram", "gemm_poly", "gemm_update"]
 MAX_NS_STEPS = 64
 
 QUINTIC = (3.4445, -4.7750, 2.0315)

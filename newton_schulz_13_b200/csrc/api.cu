@@ -53,6 +53,7 @@ int cuda_fail(cudaError_t e, const char* what) {
 // ------------------------------------------------------------------ profiling
 struct ProfRec {
   int kind;
+  int sub;     // phase class of a Newton-Schulz launch, or -1
   cudaEvent_t a, b;
   double flops, exec;
 };
@@ -72,10 +73,10 @@ cudaEvent_t get_event() {
 }
 
 template <class F>
-cudaError_t timed_launch(int kind, cudaStream_t s, double flops, double exec, F&& launch) {
+cudaError_t timed_launch(int kind, cudaStream_t s, double flops, double exec, F&& launch, int sub = -1) {
   ++g_launches;
   if (!g_prof_on) return launch();
-  ProfRec r{kind, get_event(), get_event(), flops, exec};
+  ProfRec r{kind, sub, get_event(), get_event(), flops, exec};
   cudaEventRecord(r.a, s);
   cudaError_t e = launch();
   cudaEventRecord(r.b, s);
@@ -605,11 +606,11 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
         return launch_gemm_tc_pair(static_cast<GemmProblem*>(P.d_gram[p]), n, P.tiles_gram, eg, ds.d_status, ds.pair_capacity, s);
-      });
+      }, MUON_KC_GEMM_GRAM);
     } else {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
         return launch_gemm_f32(static_cast<GemmProblemF32*>(P.d_gram[p]), n, P.tiles_gram, eg, grid * 4, s);
-      });
+      }, MUON_KC_GEMM_GRAM);
     }
     if (e != cudaSuccess) return cuda_fail(e, "gram launch");
     void* upd;
@@ -619,11 +620,11 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
       if (P.x_bf16) {
         e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
           return launch_gemm_tc_pair(static_cast<GemmProblem*>(P.d_poly), n, P.tiles_poly, ep, ds.d_status, ds.pair_capacity, s);
-        });
+        }, MUON_KC_GEMM_POLY);
       } else {
         e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
           return launch_gemm_f32(static_cast<GemmProblemF32*>(P.d_poly), n, P.tiles_poly, ep, grid * 4, s);
-        });
+        }, MUON_KC_GEMM_POLY);
       }
       if (e != cudaSuccess) return cuda_fail(e, "poly launch");
       upd = P.d_updB[p];
@@ -641,11 +642,11 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
         return launch_gemm_tc_pair(static_cast<GemmProblem*>(upd), n, P.tiles_upd, eu, ds.d_status, ds.pair_capacity, s);
-      });
+      }, MUON_KC_GEMM_UPDATE);
     } else {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
         return launch_gemm_f32(static_cast<GemmProblemF32*>(upd), n, P.tiles_upd, eu, grid * 4, s);
-      });
+      }, MUON_KC_GEMM_UPDATE);
     }
     if (e != cudaSuccess) return cuda_fail(e, "update launch");
   }
@@ -710,10 +711,13 @@ int muon_profile_read(int64_t* launches, double* ms, double* flops, double* exec
     cudaError_t e = cudaEventSynchronize(r.b);
     if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
     if (e != cudaSuccess && rc == MUON_OK) rc = cuda_fail(e, "profile event");
-    launches[r.kind] += 1;
-    ms[r.kind] += t;
-    if (flops) flops[r.kind] += r.flops;
-    if (exec_flops) exec_flops[r.kind] += r.exec;
+    for (int k : {r.kind, r.sub}) {
+      if (k < 0) continue;
+      launches[k] += 1;
+      ms[k] += t;
+      if (flops) flops[k] += r.flops;
+      if (exec_flops) exec_flops[k] += r.exec;
+    }
     g_event_pool.push_back(r.a);
     g_event_pool.push_back(r.b);
   }
