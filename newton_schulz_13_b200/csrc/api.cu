@@ -112,13 +112,12 @@ struct Shape {
 };
 
 struct BufMaps {   // TMA views of one bf16 buffer: operand loads and the epilogue's store view
-  int k128 = -1, k256 = -1, mn64 = -1, st32 = -1;
+  int k128 = -1, mn64 = -1, st32 = -1;
 };
 
 struct Plan {
   std::vector<Shape> shapes;
   int x_bf16 = 1;
-  int dev = -1;
   char* ws = nullptr;
   size_t ws_bytes = 0;
   // device tables
@@ -212,8 +211,6 @@ int device_state(DeviceState** out) {
 
 // Builds the workspace, TMA descriptors and grouped problem tables for a list of shapes.
 int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Plan** out) {
-  int dev = 0;
-  MUON_CUDA(cudaGetDevice(&dev));
   if (ds.plan && ds.plan->shapes == shapes && ds.plan->x_bf16 == x_bf16) {
     *out = ds.plan.get();
     return MUON_OK;
@@ -222,7 +219,6 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   std::unique_ptr<Plan> P(new Plan());
   P->shapes = shapes;
   P->x_bf16 = x_bf16;
-  P->dev = dev;
   const int n = (int)shapes.size();
   const size_t esz = x_bf16 ? 2 : 4;
   const size_t AL = 256;
@@ -256,7 +252,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   const size_t o_alpha = off; off = align_up(off + (size_t)n * 4, AL);
   const size_t o_part = off; off = align_up(off + (size_t)chunks * 4, AL);
   const size_t o_mats = off; off = align_up(off + (size_t)n * sizeof(MatInfo), AL);
-  const int maps_per = 16;   // 4 buffers x 4 views
+  const int maps_per = 12;   // 4 buffers x 3 views
   const size_t o_maps = off;
   if (x_bf16) off = align_up(off + (size_t)n * maps_per * sizeof(CUtensorMap), AL);
   const size_t prob_sz = x_bf16 ? sizeof(GemmProblem) : sizeof(GemmProblemF32);
@@ -305,16 +301,17 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     std::vector<CUtensorMap> maps((size_t)n * maps_per);
     CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(W + o_maps);
     int bad = 0;
-    // views: 64-wide K-major boxes of 128 or 256 rows and 64 x 64 MN-major boxes (128-byte
-    // swizzle, operand loads), and 32 x 32 boxes with the 64-byte swizzle (epilogue stores)
-    auto make4 = [&](int j, int slot, void* base, int64_t rows, int64_t cols, int64_t ld) {
+    // views: 64-wide K-major boxes of 128 rows and 64 x 64 MN-major boxes (128-byte swizzle,
+    // operand loads of one CTA of a pair), and 32 x 32 boxes with the 64-byte swizzle (epilogue
+    // loads and stores)
+    auto make3 = [&](int j, int slot, void* base, int64_t rows, int64_t cols, int64_t ld) {
       BufMaps bm;
-      const cuuint32_t bx[4] = {64u, 64u, 64u, 32u}, by[4] = {(cuuint32_t)kTcBM, (cuuint32_t)kTcBN, 64u, 32u};
-      const CUtensorMapSwizzle sw[4] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_128B,
-                                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_64B};
-      int* dst[4] = {&bm.k128, &bm.k256, &bm.mn64, &bm.st32};
-      for (int b = 0; b < 4; ++b) {
-        const int idx = j * maps_per + slot * 4 + b;
+      const cuuint32_t bx[3] = {64u, 64u, 32u}, by[3] = {(cuuint32_t)kTcBM, 64u, 32u};
+      const CUtensorMapSwizzle sw[3] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_128B,
+                                        CU_TENSOR_MAP_SWIZZLE_64B};
+      int* dst[3] = {&bm.k128, &bm.mn64, &bm.st32};
+      for (int b = 0; b < 3; ++b) {
+        const int idx = j * maps_per + slot * 3 + b;
         cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
         cuuint64_t gstride[1] = {(cuuint64_t)(ld * 2)};
         cuuint32_t box[2] = {bx[b], by[b]};
@@ -332,9 +329,9 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     for (int j = 0; j < n; ++j) {
       const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c), nn = std::max(r, c);
       const bool tall = r > c;
-      BufMaps mx[2] = {make4(j, 0, P->x0[j], r, c, P->ldx[j]), make4(j, 1, P->x1[j], r, c, P->ldx[j])};
-      BufMaps mA = make4(j, 2, P->A[j], m, m, P->ldm[j]);
-      BufMaps mB = make4(j, 3, P->B[j], m, m, P->ldm[j]);
+      BufMaps mx[2] = {make3(j, 0, P->x0[j], r, c, P->ldx[j]), make3(j, 1, P->x1[j], r, c, P->ldx[j])};
+      BufMaps mA = make3(j, 2, P->A[j], m, m, P->ldm[j]);
+      BufMaps mB = make3(j, 3, P->B[j], m, m, P->ldm[j]);
       auto M_ = [&](int idx) { return d_maps + idx; };
       for (int p = 0; p < 2; ++p) {
         GemmProblem g{};
@@ -354,9 +351,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
         g.tile_begin = tg;
         gram[p].push_back(g);
         for (int which = 0; which < 2; ++which) {   // 0: operand B, 1: operand A
-          void* S = which == 0 ? P->B[j] : P->A[j];
           const BufMaps& mS = which == 0 ? mB : mA;
-          (void)S;
           GemmProblem u{};
           if (!tall) {
             u.tma_a = M_(mS.k128); u.a_mn = 0;
@@ -381,7 +376,6 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       // B = c A A + b A (+ a I on the tensor-core path): A is symmetric, so A A = A A^T
       q.tma_a = M_(mA.k128); q.tma_b = M_(mA.k128);
       q.d = static_cast<__nv_bfloat16*>(P->B[j]); q.ldd = P->ldm[j];
-      q.c = static_cast<const __nv_bfloat16*>(P->A[j]); q.ldc = P->ldm[j];
       q.tma_d = M_(mB.st32);
       q.tma_c = M_(mA.st32);
       q.alpha = P->alpha[j];
