@@ -493,7 +493,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default="llama8b")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--e2e-group-layers", type=int, default=8,
+    ap.add_argument("--e2e-group-layers", type=int, default=4,
                     help="layers per muon_step call in the pipelined end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--sharded", action="store_true",
