@@ -331,6 +331,8 @@ def run_ours(args, world, rank, local):
         "status": status,
     }
 
+    if args.library_baseline:
+        result["library_baseline"] = run_library_baseline(args, wl, grads, stream, world, device, prof)
     if args.e2e:
         result["e2e"] = run_e2e(args, wl, step, params, grads, mom, hp, stream, world, device)
     if args.adamw:
@@ -410,6 +412,43 @@ def run_e2e(args, wl, step, params, grads, mom, hp, stream, world, device):
             "note": "grads H2D from pinned host memory and updated fp32 params D2H every step, pipelined "
                     "with the compute in groups of %d matrices (one muon_step call per group); momentum "
                     "stays resident in HBM" % (wl.count if args.sharded else per)}
+
+
+def run_library_baseline(args, wl, grads, stream, world, device, prof):
+    """Context only, not this library's path: the same Newton-Schulz iterations written with
+    torch.matmul (cuBLAS bf16 GEMMs, one matrix after another, as the pages' listing does), timed
+    on the same matrices. Compared with this library's summed Newton-Schulz launch time."""
+    import torch
+    Xs = []
+    for g in grads:
+        X = g.to(torch.bfloat16)
+        X = X / (X.float().norm() + wl.eps).to(torch.bfloat16)
+        Xs.append(X.T if X.shape[0] > X.shape[1] else X)
+
+    def ns_all():
+        for X in Xs:
+            for a, b, c in wl.coeffs:
+                A = X @ X.T
+                B = b * A + c * (A @ A)
+                X = a * X + B @ X
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            ns_all()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            ns_all()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = reduce_max(ev0.elapsed_time(ev1), world, device) / args.steps
+    ours = prof["gemm"][1] / args.steps
+    del Xs
+    torch.cuda.empty_cache()
+    return {"impl": "torch.matmul (cuBLAS), one matrix at a time", "ms_per_step": ms,
+            "nominal_tflops": wl.ns_flops() / (ms * 1e-3) / 1e12, "ours_ns_ms_per_step": ours,
+            "speedup_of_ours": ms / ours if ours else None}
 
 
 def run_adamw(args, ns, stream, world, device, hbm_peak, peak_src):
@@ -496,6 +535,9 @@ def main(argv=None):
     ap.add_argument("--e2e-group-layers", type=int, default=4,
                     help="layers per muon_step call in the pipelined end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--library-baseline", action="store_true",
+                    help="also time the same Newton-Schulz iterations written with torch.matmul (cuBLAS), "
+                         "for context")
     ap.add_argument("--sharded", action="store_true",
                     help="split one weight set across the GPUs and all-gather the updated parameters "
                          "(strong scaling) instead of one independent weight set per GPU (weak scaling)")
