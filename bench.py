@@ -236,7 +236,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream(device)
     hp = dict(lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov, weight_decay=wl.weight_decay, rms_scale=wl.rms_scale,
-              steps=len(wl.coeffs), coeffs=wl.coeffs, zero_center=wl.zero_center, eps=wl.eps, prec="bf16",
+              steps=len(wl.coeffs), coeffs=wl.coeffs, zero_center=wl.zero_center, eps=wl.eps, prec=args.prec,
               stream=stream)
 
     def step():
@@ -279,12 +279,21 @@ def run_ours(args, world, rank, local):
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     traffic = recorded_traffic()
+    fp32 = args.prec == "fp32"
+    if fp32:
+        # 3xTF32: three tf32 tensor-core products per fp32 product; the tf32 peak is the measured
+        # bf16 peak times the nominal dense ratio (1.1 / 2.25 PFLOP/s)
+        tf32_ratio = 1.1 / 2.25
+        tf32_achieved = 3.0 * achieved
+        tf32_peak = peak * tf32_ratio
+        tf32_burst = burst * tf32_ratio
     elements = wl.elements()
     gbytes = 1 if wl.grad_dtype == "bf16" else 2
     # prologue: grad + m read + m write + bf16 U write; a separate epilogue kernel (used when the
     # parameter update is not fused into the last Newton-Schulz launch): bf16 O + p read + p write
     fused_update = prof["epilogue"][0] == 0
-    ew_bytes = elements * ((2 * gbytes + 4 + 4 + 2) + (0 if fused_update else (2 + 4 + 4)))
+    xbytes = 8 if fp32 else 2   # the first iterate U: bf16, or fp32 as hi and lo tf32 planes
+    ew_bytes = elements * ((2 * gbytes + 4 + 4 + xbytes) + (0 if fused_update else (xbytes + 4 + 4)))
     ew_ms = prof["prologue"][1] + prof["epilogue"][1] + prof["norm"][1] + prof["center"][1]
     hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     ew_achieved = ew_bytes * args.steps / (ew_ms * 1e-3) / 1e9 if ew_ms > 0 else None
@@ -293,10 +302,12 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": "matrices/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if args.sharded else "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32" if fp32 else "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "matrices_per_gpu": wl.count, "elements_per_gpu": elements,
                    "grad_dtype": wl.grad_dtype, "param_dtype": "fp32", "momentum_dtype": "fp32",
                    "ns": "quintic (3.4445, -4.7750, 2.0315) x5", "lr": wl.lr, "mu": wl.mu,
+                   "ns_precision": ("fp32: 3xTF32 tensor-core products (hi/lo tf32 split), fp32 iterate"
+                                    if fp32 else "bf16 operands, fp32 accumulation"),
                    "weight_decay": wl.weight_decay, "rms_scale": "sqrt(max(1, rows/cols))",
                    "l2": "no flush: inputs (params+grads+momentum, %.0f GB per GPU) are larger than the "
                          "126 MB L2" % (elements * (4 + 4 + 2 * gbytes) / 1e9),
@@ -316,8 +327,8 @@ def run_ours(args, world, rank, local):
         "roofline_elementwise": {"bound": "hbm", "achieved": ew_achieved, "peak": hbm_peak, "unit": "GB/s",
                                  "frac": (ew_achieved / hbm_peak) if ew_achieved else None,
                                  "bytes_per_step": ew_bytes,
-                                 "bytes_definition": "per element: grad + m read + m write + bf16 U write "
-                                                     "(prologue)" + ("; the parameter update is fused into the "
+                                 "bytes_definition": "per element: grad + m read + m write + U write "
+                                                     "(bf16, or fp32 hi and lo planes) (prologue)" + ("; the parameter update is fused into the "
                                                      "last Newton-Schulz launch" if fused_update else
                                                      ", bf16 O read + p read + p write (epilogue)"),
                                  "ms_per_step": ew_ms / args.steps},
@@ -331,6 +342,18 @@ def run_ours(args, world, rank, local):
         "status": status,
     }
 
+    if fp32:
+        result["roofline"] = {
+            "bound": "tensor", "achieved": tf32_achieved, "peak": tf32_peak, "unit": "TFLOP/s",
+            "frac": tf32_achieved / tf32_peak, "traffic": None,
+            "kernel": "ns_gemm_x3_kernel (all Newton-Schulz products, 3xTF32)",
+            "peak_source": f"{peak_src} bf16_tflops_sustained x 1.1/2.25 (nominal dense tf32/bf16 ratio)",
+            "launches": g_launch, "avg_launch_ms": g_ms / max(g_launch, 1),
+            "flops_per_launch": 3.0 * g_fl / max(g_launch, 1),
+            "flops_definition": "3 tf32 products per fp32 product: 3 x (4 m^2 n + 2 m^3) per quintic "
+                                "iteration, m = min dim",
+            "fp32_equivalent_tflops": achieved, "executed_tflops": executed,
+            "frac_of_burst_peak": tf32_achieved / tf32_burst, "executed_frac": executed / tf32_peak}
     if args.library_baseline:
         result["library_baseline"] = run_library_baseline(args, wl, grads, stream, world, device, prof)
     if args.e2e:
@@ -530,6 +553,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(synth.WORKLOADS), default="llama8b")
+    ap.add_argument("--prec", choices=["bf16", "fp32"], default="bf16",
+                    help="Newton-Schulz working precision: bf16 operands (default), or fp32 through "
+                         "3xTF32 tensor-core products")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-group-layers", type=int, default=4,

@@ -61,8 +61,12 @@ typedef enum { MUON_BF16 = 0, MUON_FP32 = 1 } muon_dtype_t;
 /* Working precision of the Newton-Schulz iterate.
  *   MUON_PREC_BF16: X, A, B stored in bf16, products on tcgen05 tensor cores with fp32
  *                   accumulation (the pages' bf16 working copy).
- *   MUON_PREC_FP32: X, A, B stored in fp32, products as fp32 FMA on the CUDA cores
- *                   (a correctness mode; no speed target). */
+ *   MUON_PREC_FP32: X, A, B held in fp32, each as two planes (the value rounded toward zero to
+ *                   tf32, and the remainder); products on tcgen05 tensor cores as three tf32
+ *                   products (lo*hi + hi*lo + hi*hi, "3xTF32"), accumulated in fp32 in chunks of
+ *                   512 along K and summed in fp32 with round-to-nearest. Relative error of one
+ *                   product about 1e-6 at any K. The workspace takes 16 bytes per element of
+ *                   the iterate (bf16 mode: 4). */
 typedef enum { MUON_PREC_BF16 = 0, MUON_PREC_FP32 = 1 } muon_prec_t;
 
 /* RMS factor s of the update ("AdamW vs Muon" part 3 rescales by matrix shape without giving a

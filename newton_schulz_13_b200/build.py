@@ -9,8 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmuon.so")
-SOURCES = ["api.cu", "elementwise.cu", "ns_gemm.cu", "noalloc.cu"]
-HEADERS = ["muon_internal.h", "ptx.cuh"]
+SOURCES = ["api.cu", "elementwise.cu", "ns_gemm.cu", "ns_gemm_x3.cu", "noalloc.cu"]
+HEADERS = ["muon_internal.h", "ptx.cuh", "tile_sched.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

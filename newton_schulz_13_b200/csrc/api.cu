@@ -115,6 +115,10 @@ struct BufMaps {   // TMA views of one bf16 buffer: operand loads and the epilog
   int k128 = -1, mn64 = -1, st32 = -1;
 };
 
+struct BufMapsX3 {   // TMA views of one two-plane fp32 buffer: K-major and MN-major operand loads
+  int k128 = -1, mn32 = -1;
+};
+
 struct Plan {
   std::vector<Shape> shapes;
   int x_bf16 = 1;
@@ -144,8 +148,9 @@ struct Plan {
   // fused last update (tensor-core path): host copies of the update problems, and the per-call
   // table of the last iteration's update problems with TMA views of the caller's parameters
   std::vector<GemmProblem> h_upd[2][2];    // [operand: 0 B, 1 A][parity]
+  std::vector<GemmProblemX3> h_upd_x3[2][2];   // the same for the fp32 (3xTF32) mode
   CUtensorMap* d_pmaps = nullptr;
-  GemmProblem* d_fused = nullptr;
+  void* d_fused = nullptr;                 // GemmProblem (bf16) or GemmProblemX3 (fp32) table
   uint8_t* h_fused_pinned = nullptr;
   cudaEvent_t fused_done = nullptr;
   std::vector<uint8_t> fused_key;
@@ -183,6 +188,7 @@ struct DeviceState {
   int sms = 0;
   int cc_major = 0;
   int pair_capacity = 0;   // resident CTA pairs of the paired tensor-core kernel
+  int x3_capacity = 0;     // resident CTA pairs of the 3xTF32 kernel
 };
 
 std::map<int, DeviceState> g_dev;
@@ -201,6 +207,7 @@ int device_state(DeviceState** out) {
   if (ds.cc_major != 10)
     return fail(MUON_ERR_UNSUPPORTED, "this library runs on sm_100 (B200) devices only");
   if (ds.pair_capacity == 0) ds.pair_capacity = gemm_tc_pair_capacity(ds.sms);
+  if (ds.x3_capacity == 0) ds.x3_capacity = gemm_x3_pair_capacity(ds.sms);
   if (!ds.d_status) {
     MUON_CUDA(cudaMalloc(&ds.d_status, 2 * sizeof(int)));
     MUON_CUDA(cudaMemset(ds.d_status, 0, 2 * sizeof(int)));
@@ -220,7 +227,8 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   P->shapes = shapes;
   P->x_bf16 = x_bf16;
   const int n = (int)shapes.size();
-  const size_t esz = x_bf16 ? 2 : 4;
+  // bf16 mode: one bf16 plane per buffer; fp32 mode: hi and lo fp32 planes (GemmProblemX3)
+  const size_t esz = x_bf16 ? 2 : 8;
   const size_t AL = 256;
 
   // ---- layout
@@ -245,6 +253,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     MatInfo& mi = mats[j];
     std::memset(&mi, 0, sizeof(mi));
     mi.rows = r; mi.cols = c; mi.ldx = ldx;
+    mi.xlo = x_bf16 ? 0 : r * ldx;
     mi.chunk_begin = chunks; chunks += ceil_div(r * c, kChunk);
     mi.cs_begin = cs; cs += n_rc * n_cb;
     mi.cm_begin = cm; cm += n_cb;
@@ -252,16 +261,16 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   const size_t o_alpha = off; off = align_up(off + (size_t)n * 4, AL);
   const size_t o_part = off; off = align_up(off + (size_t)chunks * 4, AL);
   const size_t o_mats = off; off = align_up(off + (size_t)n * sizeof(MatInfo), AL);
-  const int maps_per = 12;   // 4 buffers x 3 views
+  const int maps_per = x_bf16 ? 12 : 8;   // 4 buffers x 3 views (bf16) or x 2 views (fp32)
   const size_t o_maps = off;
-  if (x_bf16) off = align_up(off + (size_t)n * maps_per * sizeof(CUtensorMap), AL);
-  const size_t prob_sz = x_bf16 ? sizeof(GemmProblem) : sizeof(GemmProblemF32);
+  off = align_up(off + (size_t)n * maps_per * sizeof(CUtensorMap), AL);
+  const size_t prob_sz = x_bf16 ? sizeof(GemmProblem) : sizeof(GemmProblemX3);
   size_t o_prob[7];
   for (int k = 0; k < 7; ++k) { o_prob[k] = off; off = align_up(off + (size_t)n * prob_sz, AL); }
   const size_t o_pmaps = off;
   if (x_bf16) off = align_up(off + (size_t)n * sizeof(CUtensorMap), AL);
   const size_t o_fused = off;
-  if (x_bf16) off = align_up(off + (size_t)n * sizeof(GemmProblem), AL);
+  off = align_up(off + (size_t)n * prob_sz, AL);
   P->ws_bytes = off;
 
   cudaError_t e = cudaMalloc(&P->ws, P->ws_bytes);
@@ -410,11 +419,38 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     P->h_upd[0][0] = updB[0]; P->h_upd[0][1] = updB[1];
     P->h_upd[1][0] = updA[0]; P->h_upd[1][1] = updA[1];
     P->d_pmaps = reinterpret_cast<CUtensorMap*>(W + o_pmaps);
-    P->d_fused = reinterpret_cast<GemmProblem*>(W + o_fused);
+    P->d_fused = W + o_fused;
     MUON_CUDA(cudaMallocHost(&P->h_fused_pinned, (size_t)n * (sizeof(CUtensorMap) + sizeof(GemmProblem))));
     MUON_CUDA(cudaEventCreateWithFlags(&P->fused_done, cudaEventDisableTiming));
   } else {
-    std::vector<GemmProblemF32> gram[2], poly, updB[2], updA[2];
+    PFN_encodeTiled_t encode = get_encode();
+    if (!encode) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    std::vector<CUtensorMap> maps((size_t)n * maps_per);
+    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(W + o_maps);
+    int bad = 0;
+    // 3-D views (columns, rows, plane) of a two-plane fp32 buffer, one plane per box: 32-wide
+    // K-major boxes of 128 rows (128-byte swizzle) and 32 x 32 MN-major boxes (128-byte swizzle
+    // over 32-byte granules, the layout tcgen05 reads MN-major tf32 operands in)
+    auto make2 = [&](int j, int slot, void* base, int64_t rows, int64_t cols, int64_t ld) {
+      BufMapsX3 bm;
+      const cuuint32_t by[2] = {(cuuint32_t)kTcBM, 32u};
+      const CUtensorMapSwizzle sw[2] = {CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B};
+      int* dst[2] = {&bm.k128, &bm.mn32};
+      for (int b = 0; b < 2; ++b) {
+        const int idx = j * maps_per + slot * 2 + b;
+        cuuint64_t gdim[3] = {(cuuint64_t)cols, (cuuint64_t)rows, 2};
+        cuuint64_t gstride[2] = {(cuuint64_t)(ld * 4), (cuuint64_t)(rows * ld * 4)};
+        cuuint32_t box[3] = {(cuuint32_t)kX3BK, by[b], 1u};
+        cuuint32_t estr[3] = {1u, 1u, 1u};
+        CUresult r = encode(&maps[idx], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, gdim, gstride, box,
+                            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw[b],
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) bad = (int)r;
+        *dst[b] = idx;
+      }
+      return bm;
+    };
+    std::vector<GemmProblemX3> gram[2], poly, updB[2], updA[2];
     uint32_t tg = 0, tp = 0, tu = 0;
     for (int j = 0; j < n; ++j) {
       const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c), nn = std::max(r, c);
@@ -423,43 +459,52 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       float* X[2] = {static_cast<float*>(P->x0[j]), static_cast<float*>(P->x1[j])};
       float* A = static_cast<float*>(P->A[j]);
       float* B = static_cast<float*>(P->B[j]);
+      BufMapsX3 mx[2] = {make2(j, 0, X[0], r, c, ldx), make2(j, 1, X[1], r, c, ldx)};
+      BufMapsX3 mA = make2(j, 2, A, m, m, ldm);
+      BufMapsX3 mB = make2(j, 3, B, m, m, ldm);
+      auto M_ = [&](int idx) { return d_maps + idx; };
       for (int p = 0; p < 2; ++p) {
-        GemmProblemF32 g{};
-        g.a = g.b = X[p];
-        if (!tall) { g.sa_i = g.sb_j = ldx; g.sa_k = g.sb_k = 1; }
-        else { g.sa_i = g.sb_j = 1; g.sa_k = g.sb_k = ldx; }
-        g.d = A; g.ldd = ldm; g.alpha = P->alpha[j];
+        GemmProblemX3 g{};
+        g.tma_a = g.tma_b = M_(tall ? mx[p].mn32 : mx[p].k128);
+        g.a_mn = g.b_mn = tall ? 1 : 0;
+        g.d = A; g.ldd = ldm; g.d_plane = m * ldm;
+        g.alpha = P->alpha[j];
         g.M = g.N = (uint32_t)m; g.K = (uint32_t)nn;
-        g.tiles_m = g.tiles_n = (uint32_t)ceil_div(m, kF32BM);
-        g.n_tiles = g.tiles_m * g.tiles_n;
+        g.tiles_m = (uint32_t)ceil_div(m, kTcPairBM); g.tiles_n = (uint32_t)ceil_div(m, kTcBN);
+        g.sym = 1;
+        g.n_tiles = (uint32_t)sym_tiles(m);
         g.tile_begin = tg;
         gram[p].push_back(g);
-        for (int which = 0; which < 2; ++which) {
-          float* S = which == 0 ? B : A;
-          GemmProblemF32 u{};
+        for (int which = 0; which < 2; ++which) {   // 0: operand B, 1: operand A
+          const BufMapsX3& mS = which == 0 ? mB : mA;
+          GemmProblemX3 u{};
           if (!tall) {
-            u.a = S; u.sa_i = ldm; u.sa_k = 1;
-            u.b = X[p]; u.sb_j = 1; u.sb_k = ldx;
+            u.tma_a = M_(mS.k128); u.a_mn = 0;
+            u.tma_b = M_(mx[p].mn32); u.b_mn = 1;
           } else {
-            u.a = X[p]; u.sa_i = ldx; u.sa_k = 1;
-            u.b = S; u.sb_j = ldm; u.sb_k = 1;
+            u.tma_a = M_(mx[p].k128); u.a_mn = 0;
+            u.tma_b = M_(mS.k128); u.b_mn = 0;
           }
-          u.d = X[1 - p]; u.ldd = ldx;
-          u.c = X[p]; u.ldc = ldx;
+          u.d = X[1 - p]; u.ldd = ldx; u.d_plane = r * ldx;
+          u.c = X[p]; u.ldc = ldx; u.c_plane = r * ldx;
           u.alpha = P->alpha[j];
           u.M = (uint32_t)r; u.N = (uint32_t)c; u.K = (uint32_t)m;
-          u.tiles_m = (uint32_t)ceil_div(r, kF32BM); u.tiles_n = (uint32_t)ceil_div(c, kF32BN);
+          u.tiles_m = (uint32_t)ceil_div(r, kTcPairBM); u.tiles_n = (uint32_t)ceil_div(c, kTcBN);
           u.n_tiles = u.tiles_m * u.tiles_n;
           u.tile_begin = tu;
           (which == 0 ? updB[p] : updA[p]).push_back(u);
         }
       }
-      GemmProblemF32 q{};
-      q.a = q.b = A; q.sa_i = q.sb_j = ldm; q.sa_k = q.sb_k = 1;
-      q.d = B; q.ldd = ldm; q.c = A; q.ldc = ldm; q.alpha = P->alpha[j];
+      GemmProblemX3 q{};
+      // B = c A A + b A: A is symmetric, so A A = A A^T
+      q.tma_a = q.tma_b = M_(mA.k128);
+      q.d = B; q.ldd = ldm; q.d_plane = m * ldm;
+      q.c = A; q.ldc = ldm; q.c_plane = m * ldm;
+      q.alpha = P->alpha[j];
       q.M = q.N = q.K = (uint32_t)m;
-      q.tiles_m = q.tiles_n = (uint32_t)ceil_div(m, kF32BM);
-      q.n_tiles = q.tiles_m * q.tiles_n;
+      q.tiles_m = (uint32_t)ceil_div(m, kTcPairBM); q.tiles_n = (uint32_t)ceil_div(m, kTcBN);
+      q.sym = 1;
+      q.n_tiles = (uint32_t)sym_tiles(m);
       q.tile_begin = tp;
       poly.push_back(q);
       tg += gram[0].back().n_tiles;
@@ -468,17 +513,28 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       P->fl_gram += 2.0 * m * m * nn;
       P->fl_poly += 2.0 * m * m * m;
       P->fl_upd += 2.0 * m * m * nn;
+      // executed: three tf32 products per tile and K step
+      const double tile_fl = 3.0 * 2.0 * kTcPairBM * kTcBN;
+      P->ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kX3BK) * kX3BK);
+      P->ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kX3BK) * kX3BK);
+      P->ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kX3BK) * kX3BK);
     }
-    P->ex_gram = P->fl_gram; P->ex_poly = P->fl_poly; P->ex_upd = P->fl_upd;
+    if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
     P->tiles_gram = tg; P->tiles_poly = tp; P->tiles_upd = tu;
-    std::vector<GemmProblemF32>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
+    MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+    std::vector<GemmProblemX3>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
                       &P->d_updA[0], &P->d_updA[1]};
     for (int k = 0; k < 7; ++k) {
       *dsts[k] = W + o_prob[k];
-      MUON_CUDA(cudaMemcpy(*dsts[k], lists[k]->data(), lists[k]->size() * sizeof(GemmProblemF32),
+      MUON_CUDA(cudaMemcpy(*dsts[k], lists[k]->data(), lists[k]->size() * sizeof(GemmProblemX3),
                            cudaMemcpyHostToDevice));
     }
+    P->h_upd_x3[0][0] = updB[0]; P->h_upd_x3[0][1] = updB[1];
+    P->h_upd_x3[1][0] = updA[0]; P->h_upd_x3[1][1] = updA[1];
+    P->d_fused = W + o_fused;
+    MUON_CUDA(cudaMallocHost(&P->h_fused_pinned, (size_t)n * sizeof(GemmProblemX3)));
+    MUON_CUDA(cudaEventCreateWithFlags(&P->fused_done, cudaEventDisableTiming));
   }
 
   // ---- per-call table staging
@@ -515,19 +571,25 @@ int upload_mats(Plan& P, std::vector<MatInfo>& mats, cudaStream_t s) {
 // or the last iteration's operand and parity change. Returns NULL when a parameter matrix cannot
 // be viewed by TMA (row length not a multiple of 4 floats, or a base not 16-byte aligned); the
 // step then uses the separate update kernel.
-const GemmProblem* fused_table(Plan& P, float* const* params, const std::vector<int>& idx,
-                               const std::vector<float>& rms, int which, int parity, cudaStream_t s,
-                               int* rc) {
-  *rc = MUON_OK;
-  const int n = (int)P.shapes.size();
-  for (int j = 0; j < n; ++j)
-    if (P.shapes[j].c % 4 != 0 || (uintptr_t)params[idx[j]] % 16 != 0) return nullptr;
+std::vector<uint8_t> fused_key_of(float* const* params, const std::vector<int>& idx,
+                                  const std::vector<float>& rms, int which, int parity) {
+  const int n = (int)idx.size();
   std::vector<uint8_t> key(sizeof(void*) * n + sizeof(float) * n + 2 * sizeof(int));
   uint8_t* k = key.data();
   for (int j = 0; j < n; ++j) { std::memcpy(k, &params[idx[j]], sizeof(void*)); k += sizeof(void*); }
   std::memcpy(k, rms.data(), sizeof(float) * n); k += sizeof(float) * n;
   std::memcpy(k, &which, sizeof(int)); k += sizeof(int);
   std::memcpy(k, &parity, sizeof(int));
+  return key;
+}
+
+const void* fused_table(Plan& P, float* const* params, const std::vector<int>& idx,
+                        const std::vector<float>& rms, int which, int parity, cudaStream_t s, int* rc) {
+  *rc = MUON_OK;
+  const int n = (int)P.shapes.size();
+  for (int j = 0; j < n; ++j)
+    if (P.shapes[j].c % 4 != 0 || (uintptr_t)params[idx[j]] % 16 != 0) return nullptr;
+  std::vector<uint8_t> key = fused_key_of(params, idx, rms, which, parity);
   if (key == P.fused_key) return P.d_fused;
   PFN_encodeTiled_t encode = get_encode();
   if (!encode) return nullptr;
@@ -559,6 +621,32 @@ const GemmProblem* fused_table(Plan& P, float* const* params, const std::vector<
   return P.d_fused;
 }
 
+// The same for the fp32 (3xTF32) mode: the epilogue updates the parameters with plain loads and
+// stores (16-byte vectors where the rows allow it), so every parameter layout is accepted.
+const void* fused_table_x3(Plan& P, float* const* params, const std::vector<int>& idx,
+                           const std::vector<float>& rms, int which, int parity, cudaStream_t s, int* rc) {
+  *rc = MUON_OK;
+  const int n = (int)P.shapes.size();
+  std::vector<uint8_t> key = fused_key_of(params, idx, rms, which, parity);
+  if (key == P.fused_key) return P.d_fused;
+  std::vector<GemmProblemX3> probs = P.h_upd_x3[which][parity];
+  for (int j = 0; j < n; ++j) {
+    float* p = params[idx[j]];
+    probs[j].p = p;
+    probs[j].ldp = P.shapes[j].c;
+    probs[j].rms = rms[j];
+    probs[j].p_vec = (P.shapes[j].c % 4 == 0 && (uintptr_t)p % 16 == 0) ? 1 : 0;
+  }
+  cudaError_t e = cudaEventSynchronize(P.fused_done);
+  if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table event"); return nullptr; }
+  std::memcpy(P.h_fused_pinned, probs.data(), n * sizeof(GemmProblemX3));
+  e = cudaMemcpyAsync(P.d_fused, P.h_fused_pinned, n * sizeof(GemmProblemX3), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaEventRecord(P.fused_done, s);
+  if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table upload"); return nullptr; }
+  P.fused_key = key;
+  return P.d_fused;
+}
+
 bool finite_f(float x) { return std::isfinite(x); }
 
 int check_coeffs(int steps, const muon_coeffs_t* coeffs, std::vector<muon_coeffs_t>& out) {
@@ -583,15 +671,15 @@ int check_shape(int64_t r, int64_t c, const char* what) {
 
 // Runs the Newton-Schulz phases for every matrix of the plan.
 int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaStream_t s,
-           const GemmProblem* fused_last = nullptr, float lr = 0.0f, float decay = 1.0f) {
+           const void* fused_last = nullptr, float lr = 0.0f, float decay = 1.0f) {
   const int n = (int)P.shapes.size();
-  const int grid = ds.sms;
   for (size_t k = 0; k < co.size(); ++k) {
     const int p = (int)(k & 1);
     const int first = k == 0 ? 1 : 0;
     const muon_coeffs_t c = co[k];
     cudaError_t e;
-    // fp32 path: gram A = alpha^2k X X^T, poly B = c A A + b A, update X' = alpha^k (a X + B X)
+    // fp32 (3xTF32) path: gram A = alpha^2k X X^T, poly B = c A A + b A,
+    //   update X' = alpha^k (a X + B X)
     //   (c = 0: X' = alpha^k (a X + b A X)).
     // bf16 path: the a X term is folded into the left operand of the update, rounding once:
     //   poly B = c A A + b A + a I (c = 0: gram A = b alpha^2k X X^T + a I), update X' = alpha^k B X.
@@ -603,7 +691,7 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
       }, MUON_KC_GEMM_GRAM);
     } else {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
-        return launch_gemm_f32(static_cast<GemmProblemF32*>(P.d_gram[p]), n, P.tiles_gram, eg, grid * 4, s);
+        return launch_gemm_x3(static_cast<GemmProblemX3*>(P.d_gram[p]), n, P.tiles_gram, eg, ds.d_status, ds.x3_capacity, s);
       }, MUON_KC_GEMM_GRAM);
     }
     if (e != cudaSuccess) return cuda_fail(e, "gram launch");
@@ -617,7 +705,7 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
         }, MUON_KC_GEMM_POLY);
       } else {
         e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
-          return launch_gemm_f32(static_cast<GemmProblemF32*>(P.d_poly), n, P.tiles_poly, ep, grid * 4, s);
+          return launch_gemm_x3(static_cast<GemmProblemX3*>(P.d_poly), n, P.tiles_poly, ep, ds.d_status, ds.x3_capacity, s);
         }, MUON_KC_GEMM_POLY);
       }
       if (e != cudaSuccess) return cuda_fail(e, "poly launch");
@@ -628,7 +716,7 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
       eu = P.x_bf16 ? EpiScalars{1.0f, 0.0f, first, 0, 0.0f} : EpiScalars{c.b, c.a, first, first, 0.0f};
     }
     if (fused_last && k + 1 == co.size()) {
-      upd = const_cast<GemmProblem*>(fused_last);
+      upd = const_cast<void*>(fused_last);
       eu.lr = lr;
       eu.decay = decay;
       eu.fused = 1;
@@ -639,7 +727,7 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
       }, MUON_KC_GEMM_UPDATE);
     } else {
       e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
-        return launch_gemm_f32(static_cast<GemmProblemF32*>(upd), n, P.tiles_upd, eu, grid * 4, s);
+        return launch_gemm_x3(static_cast<GemmProblemX3*>(upd), n, P.tiles_upd, eu, ds.d_status, ds.x3_capacity, s);
       }, MUON_KC_GEMM_UPDATE);
     }
     if (e != cudaSuccess) return cuda_fail(e, "update launch");
@@ -811,12 +899,13 @@ int muon_step(int count, float* const* params, const void* const* grads, muon_dt
   }
   rc = upload_mats(*P, mats, s);
   if (rc != MUON_OK) return rc;
-  const GemmProblem* fused = nullptr;
-  if (x_bf16 && steps > 0) {
+  const void* fused = nullptr;
+  if (steps > 0) {
     std::vector<float> rms(n);
     for (int j = 0; j < n; ++j) rms[j] = mats[j].rms;
     const int which = co.back().c != 0.0f ? 0 : 1;
-    fused = fused_table(*P, params, idx, rms, which, (steps - 1) & 1, s, &rc);
+    fused = x_bf16 ? fused_table(*P, params, idx, rms, which, (steps - 1) & 1, s, &rc)
+                   : fused_table_x3(*P, params, idx, rms, which, (steps - 1) & 1, s, &rc);
     if (rc != MUON_OK) return rc;
   }
 

@@ -77,6 +77,56 @@ __device__ __forceinline__ void store1(void* base, int64_t idx, float v) {
   else static_cast<float*>(base)[idx] = v;
 }
 
+// The Newton-Schulz iterate: bf16, or fp32 held as two planes lo_off elements apart (hi = the
+// value with its 13 low mantissa bits cleared, lo = value - hi; hi + lo is the value exactly).
+__device__ __forceinline__ float tf32_hi(float v) {
+  return __uint_as_float(__float_as_uint(v) & 0xffffe000u);
+}
+
+template <bool X_BF16>
+__device__ __forceinline__ void load8x(const void* base, int64_t idx, int64_t lo_off, float (&v)[8]) {
+  load8<X_BF16>(base, idx, v);
+  if constexpr (!X_BF16) {
+    float l[8];
+    load8<false>(base, idx + lo_off, l);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] += l[i];
+  }
+}
+
+template <bool X_BF16>
+__device__ __forceinline__ void store8x(void* base, int64_t idx, int64_t lo_off, const float (&v)[8]) {
+  if constexpr (X_BF16) {
+    store8<true>(base, idx, v);
+  } else {
+    float h[8], l[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      h[i] = tf32_hi(v[i]);
+      l[i] = v[i] - h[i];
+    }
+    store8<false>(base, idx, h);
+    store8<false>(base, idx + lo_off, l);
+  }
+}
+
+template <bool X_BF16>
+__device__ __forceinline__ float load1x(const void* base, int64_t idx, int64_t lo_off) {
+  if constexpr (X_BF16) return load1<true>(base, idx);
+  else return static_cast<const float*>(base)[idx] + static_cast<const float*>(base)[idx + lo_off];
+}
+
+template <bool X_BF16>
+__device__ __forceinline__ void store1x(void* base, int64_t idx, int64_t lo_off, float v) {
+  if constexpr (X_BF16) {
+    store1<true>(base, idx, v);
+  } else {
+    const float h = tf32_hi(v);
+    static_cast<float*>(base)[idx] = h;
+    static_cast<float*>(base)[idx + lo_off] = v - h;
+  }
+}
+
 // Deterministic block sum (fixed shuffle tree, fixed warp order).
 __device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
@@ -186,7 +236,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) prologue_kernel(const MatInfo* 
             sq += u[i] * u[i];
             bad |= !isfinite(u[i]);
           }
-          store8<X_BF16>(mi.x0, row * mi.ldx + col, u);
+          store8x<X_BF16>(mi.x0, row * mi.ldx + col, mi.xlo, u);
         }
       }
     } else if (mi.vec) {
@@ -218,7 +268,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) prologue_kernel(const MatInfo* 
           sq += u[i] * u[i];
           bad |= !isfinite(u[i]);
         }
-        store8<X_BF16>(mi.x0, row * mi.ldx + col, u);
+        store8x<X_BF16>(mi.x0, row * mi.ldx + col, mi.xlo, u);
       }
     } else {
       for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
@@ -233,7 +283,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) prologue_kernel(const MatInfo* 
         }
         sq += u * u;
         bad |= !isfinite(u);
-        store1<X_BF16>(mi.x0, row * mi.ldx + col, u);
+        store1x<X_BF16>(mi.x0, row * mi.ldx + col, mi.xlo, u);
       }
     }
     const float total = block_sum(sq, red);
@@ -282,7 +332,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) update_kernel(const MatInfo* __
         for (int q = 0; q < kBatch; ++q) {
           const int64_t e = e0 + 8 * ((int64_t)threadIdx.x + (int64_t)(b0 + q) * kEwThreads);
           const int64_t row = e / mi.cols, col = e - row * mi.cols;
-          load8<X_BF16>(mi.xf, row * mi.ldx + col, o[q]);
+          load8x<X_BF16>(mi.xf, row * mi.ldx + col, mi.xlo, o[q]);
           load8<false>(mi.p, e, p[q]);
         }
 #pragma unroll
@@ -297,7 +347,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) update_kernel(const MatInfo* __
       for (int64_t e = e0 + 8 * (int64_t)threadIdx.x; e < e1; e += 8 * (int64_t)blockDim.x) {
         const int64_t row = e / mi.cols, col = e - row * mi.cols;
         float o[8], p[8];
-        load8<X_BF16>(mi.xf, row * mi.ldx + col, o);
+        load8x<X_BF16>(mi.xf, row * mi.ldx + col, mi.xlo, o);
         load8<false>(mi.p, e, p);
 #pragma unroll
         for (int i = 0; i < 8; ++i) p[i] = p[i] * decay - step * o[i];
@@ -306,7 +356,7 @@ __global__ void __launch_bounds__(kEwThreads, 4) update_kernel(const MatInfo* __
     } else {
       for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
         const int64_t row = e / mi.cols, col = e - row * mi.cols;
-        const float o = load1<X_BF16>(mi.xf, row * mi.ldx + col);
+        const float o = load1x<X_BF16>(mi.xf, row * mi.ldx + col, mi.xlo);
         mi.p[e] = mi.p[e] * decay - step * o;
       }
     }
@@ -327,7 +377,7 @@ __global__ void __launch_bounds__(kEwThreads) output_kernel(const MatInfo* __res
       for (int64_t e = e0 + 8 * (int64_t)threadIdx.x; e < e1; e += 8 * (int64_t)blockDim.x) {
         const int64_t row = e / mi.cols, col = e - row * mi.cols;
         float o[8];
-        load8<X_BF16>(mi.xf, row * mi.ldx + col, o);
+        load8x<X_BF16>(mi.xf, row * mi.ldx + col, mi.xlo, o);
 #pragma unroll
         for (int i = 0; i < 8; ++i) o[i] *= s;
         store8<OUT_BF16>(mi.p, e, o);
@@ -335,7 +385,7 @@ __global__ void __launch_bounds__(kEwThreads) output_kernel(const MatInfo* __res
     } else {
       for (int64_t e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
         const int64_t row = e / mi.cols, col = e - row * mi.cols;
-        store1<OUT_BF16>(mi.p, e, s * load1<X_BF16>(mi.xf, row * mi.ldx + col));
+        store1<OUT_BF16>(mi.p, e, s * load1x<X_BF16>(mi.xf, row * mi.ldx + col, mi.xlo));
       }
     }
   }

@@ -32,6 +32,7 @@ struct MatInfo {
   float* alpha;        // workspace: 1 / (||u||_F + eps)
   int64_t rows, cols;  // shape of the stored matrix (row-major)
   int64_t ldx;         // leading dimension of x0 / xf, elements
+  int64_t xlo;         // fp32 workspace: offset (elements) of the low plane of x0 / xf (see below)
   int64_t chunk_begin; // first elementwise chunk of this matrix (prefix over matrices)
   int64_t cs_begin;    // first column-sum item
   int64_t cm_begin;    // first column-mean item
@@ -82,22 +83,35 @@ struct GemmProblem {
   uint8_t pad;
 };
 
-// fp32 (CUDA-core) problem: same formula, operands addressed by strides.
-struct GemmProblemF32 {
-  const float* a;   // opA(i, k) = a[i * sa_i + k * sa_k]
-  const float* b;   // opB(j, k) = b[j * sb_j + k * sb_k]
-  float* d;
-  const float* c;
-  const float* alpha;
-  int64_t sa_i, sa_k, sb_j, sb_k, ldd, ldc;
+// fp32 precision mode ("3xTF32"). Every fp32 matrix of the iteration is held as two planes of
+// the same shape and leading dimension, the second `plane` elements after the first:
+//   hi = the value with its 13 low mantissa bits cleared (exactly a tf32 number),
+//   lo = value - hi (exact in fp32),
+// so hi + lo is the value itself. One problem of a grouped 3xTF32 launch:
+//   D = s_acc * (opA . opB^T) + s_c * C + diag I,
+// with opA and opB read through 3-D TMA views (columns, rows, plane), K-major or MN-major.
+struct GemmProblemX3 {
+  const CUtensorMap* tma_a;
+  const CUtensorMap* tma_b;
+  float* d;                 // output, hi plane (the fused last update stores no D)
+  const float* c;           // addend, hi plane, or NULL
+  float* p;                 // fused last update: fp32 parameters, row stride ldp; else NULL
+  const float* alpha;       // per-matrix normalisation 1 / (||u|| + eps)
+  int64_t ldd, ldc, ldp;
+  int64_t d_plane, c_plane; // offset (elements) of the lo plane of d and of c
   uint32_t M, N, K;
-  uint32_t tiles_m, tiles_n, tile_begin, n_tiles;
-  uint32_t sym;
+  uint32_t tiles_m, tiles_n;
+  uint32_t tile_begin;
+  uint32_t n_tiles;
+  float rms;                // fused last update: RMS factor s of this matrix
+  uint8_t a_mn, b_mn;       // 1: operand is MN-major
+  uint8_t sym;              // 1: D is symmetric (upper-triangle tiles, strictly-upper part mirrored)
+  uint8_t p_vec;            // 1: p rows are 16-byte aligned (ldp % 4 == 0, p 16-byte aligned)
 };
 
 // Epilogue scalars of one launch: D = k_acc alpha^e_acc acc + k_c alpha^e_c C + diag I
-// (diag is applied by the CTA-pair kernel only, on symmetric outputs). With fused set (CTA-pair
-// kernel, last Newton-Schulz update), O = k_acc alpha^e_acc acc is not stored; instead the
+// (diag is applied by the CTA-pair kernels only; the bf16 CTA-pair kernel takes alpha^e_c = 1).
+// With fused set (CTA-pair kernels, last Newton-Schulz update), O = D is not stored; instead the
 // parameters become p (1 - lr wd) - lr s O, with decay = 1 - lr wd and s = rms of the problem.
 struct EpiScalars {
   float k_acc, k_c;
@@ -126,8 +140,9 @@ cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_
 cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                 EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
 int gemm_tc_pair_capacity(int sms);
-cudaError_t launch_gemm_f32(const GemmProblemF32* probs, int nprobs, uint32_t total_tiles,
-                            EpiScalars ep, int grid, cudaStream_t s);
+cudaError_t launch_gemm_x3(const GemmProblemX3* probs, int nprobs, uint32_t total_tiles,
+                           EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
+int gemm_x3_pair_capacity(int sms);
 
 // Tile geometry of the tensor-core kernel: single-CTA tiles are kTcBM x kTcBN, CTA-pair tiles
 // kTcPairBM x kTcBN; K advances kTcBK per pipeline stage.
@@ -135,8 +150,8 @@ constexpr int kTcBM = 128;
 constexpr int kTcPairBM = 256;
 constexpr int kTcBN = 256;
 constexpr int kTcBK = 64;
-// Tile geometry of the fp32 kernel.
-constexpr int kF32BM = 64;
-constexpr int kF32BN = 64;
+// 3xTF32 kernel: CTA-pair tiles kTcPairBM x kTcBN, K advances kX3BK (one 128-byte row of fp32)
+// per pipeline stage.
+constexpr int kX3BK = 32;
 
 }  // namespace muon

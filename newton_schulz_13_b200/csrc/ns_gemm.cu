@@ -27,6 +27,7 @@
 
 #include "muon_internal.h"
 #include "ptx.cuh"
+#include "tile_sched.cuh"
 
 namespace muon {
 namespace {
@@ -34,7 +35,6 @@ namespace {
 constexpr uint32_t kBoxBytes = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 M/N columns
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
-constexpr uint32_t kGroupM = 8;
 
 // Geometry of the two variants. Each CTA owns 128 accumulator rows x 256 columns (two
 // accumulators = all 512 tensor-memory columns).
@@ -62,53 +62,6 @@ struct TcCfg {
 // 64-byte swizzle the TMA store expects (chunk index XOR bits 1-2 of the row).
 __device__ __forceinline__ uint32_t sw64_chunk(uint32_t r, uint32_t j) {
   return r * 64u + ((j ^ ((r >> 1) & 3u)) << 4);
-}
-
-struct Tile {
-  int p;
-  uint32_t bi, bj;
-};
-
-template <int TILE_M, int TILE_N>
-__device__ __forceinline__ Tile decode_tile(const GemmProblem* __restrict__ probs, int nprobs,
-                                            uint32_t t) {
-  int lo = 0, hi = nprobs - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (probs[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
-  }
-  const GemmProblem& P = probs[lo];
-  uint32_t l = t - P.tile_begin;
-  Tile tl;
-  tl.p = lo;
-  if (P.sym) {
-    // row block bi covers rows [TILE_M bi, TILE_M (bi + 1)); its first column block touching the
-    // upper triangle is (TILE_M bi) / TILE_N.
-    uint32_t bi = 0;
-    while (true) {
-      const uint32_t first = (bi * TILE_M) / TILE_N;
-      const uint32_t cnt = P.tiles_n - first;
-      if (l < cnt) { tl.bi = bi; tl.bj = first + l; break; }
-      l -= cnt;
-      ++bi;
-    }
-  } else {
-    // grouped raster: kGroupM row blocks sweep all column blocks together (L2 reuse)
-    const uint32_t per_group = kGroupM * P.tiles_n;
-    const uint32_t g = l / per_group;
-    const uint32_t first = g * kGroupM;
-    const uint32_t gsize = min(kGroupM, P.tiles_m - first);
-    const uint32_t r = l - g * per_group;
-    tl.bi = first + r % gsize;
-    tl.bj = r / gsize;
-  }
-  return tl;
-}
-
-__device__ __forceinline__ float alpha_pow(float alpha, int e) {
-  float s = 1.0f;
-  for (int i = 0; i < e; ++i) s *= alpha;
-  return s;
 }
 
 template <bool PAIR>
@@ -526,66 +479,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// ---------------------------------------------------------------- fp32 CUDA-core variant
-constexpr int kF32BK = 16;
-
-__global__ void __launch_bounds__(256)
-    ns_gemm_f32_kernel(const GemmProblemF32* __restrict__ probs, int nprobs, uint32_t total_tiles,
-                       EpiScalars ep) {
-  __shared__ float As[kF32BK][kF32BM + 4];
-  __shared__ float Bs[kF32BK][kF32BN + 4];
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  for (uint32_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-    int lo = 0, hi = nprobs - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (probs[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
-    }
-    const GemmProblemF32& P = probs[lo];
-    const uint32_t l = t - P.tile_begin;
-    const int64_t i0 = (int64_t)(l / P.tiles_n) * kF32BM, j0 = (int64_t)(l % P.tiles_n) * kF32BN;
-    float acc[4][4] = {};
-    for (int64_t k0 = 0; k0 < P.K; k0 += kF32BK) {
-      for (int e = threadIdx.x; e < kF32BK * kF32BM; e += blockDim.x) {
-        const int kk = e / kF32BM, ii = e % kF32BM;
-        const int64_t gi = i0 + ii, gk = k0 + kk;
-        As[kk][ii] = (gi < P.M && gk < P.K) ? P.a[gi * P.sa_i + gk * P.sa_k] : 0.0f;
-        const int64_t gj = j0 + ii;
-        Bs[kk][ii] = (gj < P.N && gk < P.K) ? P.b[gj * P.sb_j + gk * P.sb_k] : 0.0f;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int kk = 0; kk < kF32BK; ++kk) {
-        float a[4], b[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          a[x] = As[kk][ty * 4 + x];
-          b[x] = Bs[kk][tx * 4 + x];
-        }
-#pragma unroll
-        for (int x = 0; x < 4; ++x)
-#pragma unroll
-          for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(a[x], b[y], acc[x][y]);
-      }
-      __syncthreads();
-    }
-    const float alpha = (ep.e_acc | ep.e_c) ? *P.alpha : 1.0f;
-    const float s_acc = ep.k_acc * alpha_pow(alpha, ep.e_acc);
-    const float s_c = ep.k_c * alpha_pow(alpha, ep.e_c);
-    for (int x = 0; x < 4; ++x) {
-      const int64_t gi = i0 + ty * 4 + x;
-      if (gi >= P.M) continue;
-      for (int y = 0; y < 4; ++y) {
-        const int64_t gj = j0 + tx * 4 + y;
-        if (gj >= P.N) continue;
-        float v = s_acc * acc[x][y];
-        if (P.c != nullptr && s_c != 0.0f) v += s_c * P.c[gi * P.ldc + gj];
-        P.d[gi * P.ldd + gj] = v;
-      }
-    }
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
@@ -656,14 +549,5 @@ int gemm_tc_pair_capacity(int sms) {
   }
   return n;
 }
-
-cudaError_t launch_gemm_f32(const GemmProblemF32* probs, int nprobs, uint32_t total_tiles,
-                            EpiScalars ep, int grid, cudaStream_t s) {
-  if (total_tiles == 0) return cudaSuccess;
-  if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
-  ns_gemm_f32_kernel<<<grid, 256, 0, s>>>(probs, nprobs, total_tiles, ep);
-  return cudaGetLastError();
-}
-
 
 }  // namespace muon

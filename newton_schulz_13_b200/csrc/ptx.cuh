@@ -114,6 +114,17 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorM
       : "memory");
 }
 
+// 3-D paired-CTA form (x innermost, then y, then z), used for the two-plane fp32 buffers: z
+// selects the plane.
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int32_t x, int32_t y,
+                                                 int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 // ---- TMA stores from shared memory (bulk async-group completion)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -232,6 +243,17 @@ __device__ __forceinline__ void tc_mma_f16_pair(uint32_t d_tmem, uint64_t a_desc
       : "memory");
 }
 
+// kind::tf32: A and B are 32-bit words of which the tensor core uses the tf32 part (sign, 8-bit
+// exponent, 10 mantissa bits); fp32 accumulation.
+__device__ __forceinline__ void tc_mma_tf32_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrives once on the mbarrier at this offset in every CTA of `cta_mask` when all previously
 // issued paired MMAs of this thread have completed.
 __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_mask) {
@@ -252,9 +274,10 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
 // Shared-memory matrix descriptor for tcgen05.mma with the 128-byte swizzle:
 //   bits  0-13 start address >> 4, 16-29 leading byte offset >> 4, 32-45 stride byte offset >> 4,
 //   bits 46-47 descriptor version (1), 49-51 base offset (0), 61-63 layout (2 = 128B swizzle).
-// K-major operand: rows of 128 bytes (64 bf16 along K), 8-row groups SBO = 1024 bytes apart.
+// K-major operand: rows of 128 bytes (64 bf16 or 32 tf32 along K), 8-row groups SBO = 1024
+// bytes apart.
 // MN-major operand: rows of 128 bytes along M/N (64 elements), one row per K index,
-//   8-row (K) groups SBO apart, 64-element M/N blocks LBO apart.
+//   8-row (K) groups SBO apart, 128-byte M/N blocks (64 bf16 or 32 tf32) LBO apart.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_addr, uint32_t lbo_bytes,
                                                     uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -266,12 +289,29 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_addr, uint32_t
   return d;
 }
 
+// The same with layout 1, the 128-byte swizzle over 32-byte granules (granule index XOR bits 0-1
+// of the 128-byte row index, repeating every 4 rows), the form tcgen05 reads MN-major tf32
+// operands in: rows of 128 bytes along M/N (32 tf32), 4-row (K) groups SBO apart, 128-byte M/N
+// blocks LBO apart. TMA writes this layout with CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B.
+__device__ __forceinline__ uint64_t smem_desc_sw128_atom32(uint32_t smem_addr, uint32_t lbo_bytes,
+                                                           uint32_t sbo_bytes) {
+  return (smem_desc_sw128(smem_addr, lbo_bytes, sbo_bytes) & ~(7ull << 61)) | (1ull << 61);
+}
+
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 D, dense:
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16),
 //   bit 15 A major (1 = MN), bit 16 B major (1 = MN), bits 17-22 N >> 3, bits 24-28 M >> 4.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, uint32_t a_mn,
                                                        uint32_t b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn << 15) | (b_mn << 16) | ((N >> 3) << 17) |
+         ((M >> 4) << 24);
+}
+
+// Instruction descriptor, kind::tf32 with tf32 A and B (format code 2), fp32 D, dense; the other
+// fields as in idesc_bf16_f32.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(uint32_t M, uint32_t N, uint32_t a_mn,
+                                                       uint32_t b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | (a_mn << 15) | (b_mn << 16) | ((N >> 3) << 17) |
          ((M >> 4) << 24);
 }
 

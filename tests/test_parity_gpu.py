@@ -68,17 +68,49 @@ def test_ns_orthogonalize_fp32(shape, sched):
 
 @pytest.mark.parametrize("shape", [(1 << 20, 16), (16, 1 << 20), (2, 1 << 20)], ids=lambda s: f"{s[0]}x{s[1]}")
 @pytest.mark.parametrize("sched", ["quintic5", "cubic5"], ids=str)
-def test_ns_largest_single_dimension(shape, sched):
+@pytest.mark.parametrize("prec,tol", [("bf16", TOL_O_BF16), ("fp32", TOL_O_FP32)], ids=["bf16", "fp32"])
+def test_ns_largest_single_dimension(shape, sched, prec, tol):
     """The largest row or column count the C ABI accepts (2^20), on thin matrices the oracle still
     finishes in a second: Gram contractions over a million-long K, 4096 row tiles of the update."""
     import newton_schulz_13_b200 as ns
     co = SCHEDULES[sched]
     G = synth.round_to(_gen(shape, 17), "bf16")
-    X = ns.ns_orthogonalize(to_dev(G, torch.bfloat16), steps=len(co), coeffs=co, eps=1e-7, prec="bf16",
+    X = ns.ns_orthogonalize(to_dev(G, torch.bfloat16), steps=len(co), coeffs=co, eps=1e-7, prec=prec,
                             out_dtype=torch.float32)
     assert ns.check_status() == ns.OK
     want = oracle.newton_schulz(G, co, eps=1e-7)
-    assert rel(host64(X), want) <= TOL_O_BF16, rel(host64(X), want)
+    assert rel(host64(X), want) <= tol, rel(host64(X), want)
+
+
+@pytest.mark.parametrize("shape", [(33, 17), (300, 701), (701, 300), (520, 520)], ids=lambda s: f"{s[0]}x{s[1]}")
+@pytest.mark.parametrize("offset", [0, 1], ids=["aligned", "offset1"])
+def test_step_fp32_mode_ragged_and_unaligned_params(shape, offset):
+    """fp32 mode fuses the parameter update into the last Newton-Schulz product with plain loads and
+    stores: rows whose length is not a multiple of 4 floats, and parameter matrices that start one
+    float past a 16-byte boundary, take the scalar path of that epilogue."""
+    import newton_schulz_13_b200 as ns
+    r, c = shape
+    rng = np.random.default_rng(23)
+    p0 = synth.round_to(0.02 * rng.standard_normal((r, c)), "fp32")
+    g = synth.round_to(rng.standard_normal((r, c)), "fp32")
+    store = torch.zeros(r * c + offset, dtype=torch.float32, device="cuda")
+    p = store[offset:].view(r, c)
+    p.copy_(torch.from_numpy(p0))
+    m = torch.zeros((r, c), dtype=torch.float32, device="cuda")
+    lr, wd = 0.02, 0.1
+    ns.muon_step([p], [to_dev(g, torch.float32)], [m], lr=lr, mu=0.95, nesterov=True, weight_decay=wd,
+                 rms_scale=1, steps=5, coeffs=Q5, eps=1e-7, prec="fp32")
+    torch.cuda.synchronize()
+    assert ns.check_status() == ns.OK
+    o_p, o_m = p0.astype(np.float64).copy(), np.zeros((r, c))
+    O_ref = oracle.muon_step([o_p], [g], [o_m], lr=lr, mu=0.95, nesterov=True, weight_decay=wd,
+                             rms_mode=1, coeffs=Q5, zero_center=False, eps=1e-7, want_O=True)[0]
+    s = np.sqrt(max(1.0, r / c))
+    decay = np.float64(np.float32(1.0 - np.float32(lr) * np.float32(wd)))
+    O_gpu = (p0 * decay - host64(p)) / (np.float64(np.float32(lr)) * s)
+    assert rel(O_gpu, O_ref) <= TOL_O_FP32, rel(O_gpu, O_ref)
+    assert rel(host64(p), o_p) <= TOL_P
+    assert rel(host64(m), o_m) <= TOL_M
 
 
 @pytest.mark.parametrize("shape", [(96, 200), (200, 96), (64, 64)], ids=lambda s: f"{s[0]}x{s[1]}")

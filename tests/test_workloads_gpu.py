@@ -96,6 +96,23 @@ def test_mamba_24_three_steps():
     run_and_check(StepCase(wl, sample=[0, 1, 2, 3, 93, 94], device_fill=True), wl.n_steps)
 
 
+def test_gpt2_small_fp32_mode_two_steps():
+    wl = synth.WORKLOADS["gpt2_small"]
+    run_and_check(StepCase(wl, sample=[0, 1, 3, 45], device_fill=True), 2, prec="fp32", tol_o=TOL_O_FP32)
+
+
+def test_mamba_24_fp32_mode_three_steps():
+    wl = synth.WORKLOADS["mamba_24"]
+    run_and_check(StepCase(wl, sample=[0, 1, 2, 3, 93, 94], device_fill=True), wl.n_steps, prec="fp32",
+                  tol_o=TOL_O_FP32)
+
+
+def test_llama8b_layer_fp32_mode():
+    wl = synth.WORKLOADS["llama8b_layer"]
+    # Wk, Wv (1024 x 4096): the oracle's full step finishes in seconds
+    run_and_check(StepCase(wl, sample=[1, 2], device_fill=True), 1, prec="fp32", tol_o=TOL_O_FP32)
+
+
 # ----------------------------------------------------------------------------- Llama-8B, full size
 def _top_triplets(X: np.ndarray, k: int = 6, iters: int = 80, seed: int = 0):
     """Top-k singular triplets of X by block power iteration with a final Rayleigh-Ritz step."""
