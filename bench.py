@@ -35,7 +35,8 @@ import synth  # noqa: E402
 METRIC = "Muon step matrices/s and NS TFLOP/s (bf16) vs B200 dense tensor peak, 1 GPU"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ns_gemm_tc_llama8b_traffic.txt")
-KERNEL_SOURCES = [os.path.join(ROOT, "newton_schulz_13_b200", "csrc", f) for f in ("ns_gemm.cu", "ptx.cuh")]
+KERNEL_SOURCES = [os.path.join(ROOT, "newton_schulz_13_b200", "csrc", f)
+                  for f in ("ns_gemm.cu", "ptx.cuh", "tile_sched.cuh")]
 KERNEL_HEADER = os.path.join(ROOT, "newton_schulz_13_b200", "csrc", "muon_internal.h")
 
 
@@ -51,16 +52,17 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    """Hash of the tensor-core kernel's source: its .cu file, the PTX helpers and, from the shared
-    header, the problem and epilogue structures it reads (other declarations there do not count)."""
+    """Hash of the bf16 tensor-core kernel's source: its .cu file, the PTX helpers, the tile
+    schedule and, from the shared header, the two structures it reads (GemmProblem, EpiScalars);
+    other declarations there do not count."""
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
         with open(p, "rb") as f:
             h.update(f.read())
     text = open(KERNEL_HEADER).read()
-    start = text.index("struct GemmProblem {")
-    end = text.index("};", text.index("struct EpiScalars {")) + 2
-    h.update(text[start:end].encode())
+    for name in ("struct GemmProblem {", "struct EpiScalars {"):
+        start = text.index(name)
+        h.update(text[start:text.index("};", start) + 2].encode())
     return h.hexdigest()[:16]
 
 
