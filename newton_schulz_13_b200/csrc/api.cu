@@ -102,6 +102,11 @@ PFN_encodeTiled_t get_encode() {
   return fn;
 }
 
+// Per-call tables are written in 8-byte words (write_table).
+static_assert(sizeof(MatInfo) % 8 == 0 && sizeof(AdamTensor) % 8 == 0, "table rows are 8-byte words");
+static_assert(sizeof(GemmProblem) % 8 == 0 && sizeof(GemmProblemX3) % 8 == 0, "table rows are 8-byte words");
+static_assert(sizeof(CUtensorMap) % 8 == 0, "table rows are 8-byte words");
+
 // ------------------------------------------------------------------ plan
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -140,10 +145,8 @@ struct Plan {
   uint32_t tiles_gram = 0, tiles_poly = 0, tiles_upd = 0;
   double fl_gram = 0, fl_poly = 0, fl_upd = 0;      // nominal flops per launch
   double ex_gram = 0, ex_poly = 0, ex_upd = 0;      // executed (tile) flops per launch
-  // per-call MatInfo staging
+  // per-call MatInfo table (written through kernel parameters when it changes)
   std::vector<MatInfo> last_uploaded;
-  MatInfo* h_pinned = nullptr;
-  cudaEvent_t upload_done = nullptr;
   bool uploaded_once = false;
   // fused last update (tensor-core path): host copies of the update problems, and the per-call
   // table of the last iteration's update problems with TMA views of the caller's parameters
@@ -151,32 +154,22 @@ struct Plan {
   std::vector<GemmProblemX3> h_upd_x3[2][2];   // the same for the fp32 (3xTF32) mode
   CUtensorMap* d_pmaps = nullptr;
   void* d_fused = nullptr;                 // GemmProblem (bf16) or GemmProblemX3 (fp32) table
-  uint8_t* h_fused_pinned = nullptr;
-  cudaEvent_t fused_done = nullptr;
   std::vector<uint8_t> fused_key;
 
   ~Plan() {
-    if (fused_done) cudaEventDestroy(fused_done);
-    if (h_fused_pinned) cudaFreeHost(h_fused_pinned);
-    if (upload_done) cudaEventDestroy(upload_done);
-    if (h_pinned) cudaFreeHost(h_pinned);
     if (ws) cudaFree(ws);
   }
 };
 
-// Per-device table of an AdamW call: one AdamTensor per tensor, re-uploaded (from pinned staging)
-// only when the pointers change.
+// Per-device table of an AdamW call: one AdamTensor per tensor, rewritten (through kernel
+// parameters) only when the pointers change.
 struct AdamPlan {
   std::vector<int64_t> numel;
   AdamTensor* d_tab = nullptr;
-  AdamTensor* h_pinned = nullptr;
-  cudaEvent_t done = nullptr;
   std::vector<AdamTensor> last;
   bool uploaded = false;
   int64_t n_chunks = 0;
   ~AdamPlan() {
-    if (done) cudaEventDestroy(done);
-    if (h_pinned) cudaFreeHost(h_pinned);
     if (d_tab) cudaFree(d_tab);
   }
 };
@@ -420,8 +413,6 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     P->h_upd[1][0] = updA[0]; P->h_upd[1][1] = updA[1];
     P->d_pmaps = reinterpret_cast<CUtensorMap*>(W + o_pmaps);
     P->d_fused = W + o_fused;
-    MUON_CUDA(cudaMallocHost(&P->h_fused_pinned, (size_t)n * (sizeof(CUtensorMap) + sizeof(GemmProblem))));
-    MUON_CUDA(cudaEventCreateWithFlags(&P->fused_done, cudaEventDisableTiming));
   } else {
     PFN_encodeTiled_t encode = get_encode();
     if (!encode) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
@@ -533,13 +524,9 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     P->h_upd_x3[0][0] = updB[0]; P->h_upd_x3[0][1] = updB[1];
     P->h_upd_x3[1][0] = updA[0]; P->h_upd_x3[1][1] = updA[1];
     P->d_fused = W + o_fused;
-    MUON_CUDA(cudaMallocHost(&P->h_fused_pinned, (size_t)n * sizeof(GemmProblemX3)));
-    MUON_CUDA(cudaEventCreateWithFlags(&P->fused_done, cudaEventDisableTiming));
   }
 
-  // ---- per-call table staging
-  MUON_CUDA(cudaMallocHost(&P->h_pinned, (size_t)n * sizeof(MatInfo)));
-  MUON_CUDA(cudaEventCreateWithFlags(&P->upload_done, cudaEventDisableTiming));
+  // ---- per-call table template
   for (int j = 0; j < n; ++j) {
     mats[j].x0 = P->x0[j];
     mats[j].colmean = P->colmean[j];
@@ -552,14 +539,12 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   return MUON_OK;
 }
 
-// Fills the per-call fields and uploads the table when it differs from the last upload.
+// Writes the per-call table when it differs from the last one written (in stream order, through
+// kernel parameters).
 int upload_mats(Plan& P, std::vector<MatInfo>& mats, cudaStream_t s) {
   if (P.uploaded_once && std::memcmp(mats.data(), P.last_uploaded.data(), mats.size() * sizeof(MatInfo)) == 0)
     return MUON_OK;
-  MUON_CUDA(cudaEventSynchronize(P.upload_done));
-  std::memcpy(P.h_pinned, mats.data(), mats.size() * sizeof(MatInfo));
-  MUON_CUDA(cudaMemcpyAsync(P.d_mats, P.h_pinned, mats.size() * sizeof(MatInfo), cudaMemcpyHostToDevice, s));
-  MUON_CUDA(cudaEventRecord(P.upload_done, s));
+  MUON_CUDA(write_table(P.d_mats, mats.data(), mats.size() * sizeof(MatInfo), s, &g_launches));
   P.last_uploaded = mats;
   P.uploaded_once = true;
   return MUON_OK;
@@ -607,15 +592,8 @@ const void* fused_table(Plan& P, float* const* params, const std::vector<int>& i
     probs[j].tma_p = P.d_pmaps + j;
     probs[j].rms = rms[j];
   }
-  cudaError_t e = cudaEventSynchronize(P.fused_done);
-  if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table event"); return nullptr; }
-  std::memcpy(P.h_fused_pinned, maps.data(), n * sizeof(CUtensorMap));
-  std::memcpy(P.h_fused_pinned + n * sizeof(CUtensorMap), probs.data(), n * sizeof(GemmProblem));
-  e = cudaMemcpyAsync(P.d_pmaps, P.h_fused_pinned, n * sizeof(CUtensorMap), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(P.d_fused, P.h_fused_pinned + n * sizeof(CUtensorMap), n * sizeof(GemmProblem),
-                        cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaEventRecord(P.fused_done, s);
+  cudaError_t e = write_table(P.d_pmaps, maps.data(), n * sizeof(CUtensorMap), s, &g_launches);
+  if (e == cudaSuccess) e = write_table(P.d_fused, probs.data(), n * sizeof(GemmProblem), s, &g_launches);
   if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table upload"); return nullptr; }
   P.fused_key = key;
   return P.d_fused;
@@ -637,11 +615,7 @@ const void* fused_table_x3(Plan& P, float* const* params, const std::vector<int>
     probs[j].rms = rms[j];
     probs[j].p_vec = (P.shapes[j].c % 4 == 0 && (uintptr_t)p % 16 == 0) ? 1 : 0;
   }
-  cudaError_t e = cudaEventSynchronize(P.fused_done);
-  if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table event"); return nullptr; }
-  std::memcpy(P.h_fused_pinned, probs.data(), n * sizeof(GemmProblemX3));
-  e = cudaMemcpyAsync(P.d_fused, P.h_fused_pinned, n * sizeof(GemmProblemX3), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaEventRecord(P.fused_done, s);
+  cudaError_t e = write_table(P.d_fused, probs.data(), n * sizeof(GemmProblemX3), s, &g_launches);
   if (e != cudaSuccess) { *rc = cuda_fail(e, "fused table upload"); return nullptr; }
   P.fused_key = key;
   return P.d_fused;
@@ -976,8 +950,6 @@ int muon_adamw_step(int count, float* const* params, const void* const* grads, m
     std::unique_ptr<AdamPlan> A(new AdamPlan());
     A->numel = nel;
     MUON_CUDA(cudaMalloc(&A->d_tab, (size_t)n * sizeof(AdamTensor)));
-    MUON_CUDA(cudaMallocHost(&A->h_pinned, (size_t)n * sizeof(AdamTensor)));
-    MUON_CUDA(cudaEventCreateWithFlags(&A->done, cudaEventDisableTiming));
     ds->adam = std::move(A);
   }
   AdamPlan& A = *ds->adam;
@@ -999,10 +971,7 @@ int muon_adamw_step(int count, float* const* params, const void* const* grads, m
   }
   A.n_chunks = chunks;
   if (!A.uploaded || std::memcmp(tab.data(), A.last.data(), n * sizeof(AdamTensor)) != 0) {
-    MUON_CUDA(cudaEventSynchronize(A.done));
-    std::memcpy(A.h_pinned, tab.data(), n * sizeof(AdamTensor));
-    MUON_CUDA(cudaMemcpyAsync(A.d_tab, A.h_pinned, n * sizeof(AdamTensor), cudaMemcpyHostToDevice, s));
-    MUON_CUDA(cudaEventRecord(A.done, s));
+    MUON_CUDA(write_table(A.d_tab, tab.data(), n * sizeof(AdamTensor), s, &g_launches));
     A.last = tab;
     A.uploaded = true;
   }

@@ -15,6 +15,11 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <algorithm>
+#include <cstring>
+#include <memory>
+
+
 #include "muon_internal.h"
 
 namespace muon {
@@ -140,6 +145,11 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   }
   __syncthreads();
   return s;
+}
+
+// ---------------------------------------------------------------- per-call tables
+__global__ void __launch_bounds__(256) table_write_kernel(const __grid_constant__ TableChunk c) {
+  for (uint64_t i = threadIdx.x; i < c.nwords; i += blockDim.x) c.dst[i] = c.w[i];
 }
 
 // ---------------------------------------------------------------- zero-centring
@@ -476,6 +486,24 @@ cudaError_t launch_colsum(const MatInfo* mats, int nmats, int64_t items, int g_b
   if (g_bf16) colsum_kernel<true><<<grid, kCsCols, 0, s>>>(mats, nmats, items);
   else colsum_kernel<false><<<grid, kCsCols, 0, s>>>(mats, nmats, items);
   return cudaGetLastError();
+}
+
+cudaError_t write_table(void* dst, const void* src, size_t bytes, cudaStream_t s, int64_t* launches) {
+  if (bytes % 8 != 0) return cudaErrorInvalidValue;
+  thread_local std::unique_ptr<TableChunk> chunk(new TableChunk());
+  const uint64_t* words = static_cast<const uint64_t*>(src);
+  const size_t total = bytes / 8;
+  for (size_t off = 0; off < total; off += kTableWords) {
+    const size_t n = std::min<size_t>(kTableWords, total - off);
+    chunk->dst = static_cast<uint64_t*>(dst) + off;
+    chunk->nwords = n;
+    std::memcpy(chunk->w, words + off, n * 8);
+    table_write_kernel<<<1, 256, 0, s>>>(*chunk);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (launches) ++*launches;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_colmean(const MatInfo* mats, int nmats, int64_t items, cudaStream_t s) {

@@ -121,7 +121,20 @@ struct EpiScalars {
   int fused;
 };
 
+// Per-call tables (pointer tables of a call) travel to the device inside kernel parameters, not
+// through a copy engine: a small copy on the caller's stream would otherwise queue behind whatever
+// bulk copies the caller has in flight (up to the whole step's gradient upload).
+constexpr int kTableWords = 4000;   // 32,000 bytes of payload per launch (parameter limit 32,764)
+struct TableChunk {
+  uint64_t* dst;
+  uint64_t nwords;
+  uint64_t w[kTableWords];
+};
+
 // ---- launchers (defined in the .cu files) ----
+// Writes `bytes` (a multiple of 8) from host memory to device memory at dst, in stream order, with
+// ceil(bytes / 32000) launches of a copy kernel; adds the number of launches to *launches.
+cudaError_t write_table(void* dst, const void* src, size_t bytes, cudaStream_t s, int64_t* launches);
 cudaError_t launch_colsum(const MatInfo* mats, int nmats, int64_t items, int g_bf16, cudaStream_t s);
 cudaError_t launch_colmean(const MatInfo* mats, int nmats, int64_t items, cudaStream_t s);
 cudaError_t launch_prologue(const MatInfo* mats, int nmats, int64_t chunks, int g_bf16, int x_bf16,

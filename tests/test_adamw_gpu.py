@@ -83,3 +83,30 @@ def test_edge_cases_ragged_misaligned_skipped():
         assert rel(host64(ms[i]), o_m[i]) <= TOL or not o_m[i].any()
     assert torch.equal(ms[2], torch.zeros_like(ms[2]))
     assert np.array_equal(host64(ps[2]), p0[2].astype(np.float32).astype(np.float64))
+
+
+def test_many_tensors_multi_chunk_table():
+    """1,000 tensors: the AdamW tensor table exceeds one 32,000-byte kernel-parameter chunk and is
+    written in several launches; every tensor is checked."""
+    import newton_schulz_13_b200 as ns
+    rng = np.random.default_rng(5)
+    sizes = [1 + 37 * (i % 11) for i in range(1000)]
+    p0 = [rng.standard_normal(n).astype(np.float32) for n in sizes]
+    g = [rng.standard_normal(n).astype(np.float32) for n in sizes]
+    ps = [to_dev(x, torch.float32) for x in p0]
+    ms = [torch.zeros(n, device="cuda") for n in sizes]
+    vs = [torch.zeros(n, device="cuda") for n in sizes]
+    # the C ABI takes the hyper-parameters as floats: the oracle gets the same fp32 values (with
+    # beta2 = 0.999, 1 - fp32(beta2) differs from 0.001 by 1.3e-5 relative, and so does v)
+    hp = {k: float(np.float32(v)) for k, v in
+          dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.01).items()}
+    ns.adamw_step(ps, [to_dev(x, torch.float32) for x in g], ms, vs, step=1, **hp)
+    o_p = [x.astype(np.float64) for x in p0]
+    o_m = [np.zeros(n) for n in sizes]
+    o_v = [np.zeros(n) for n in sizes]
+    oracle.adamw_step(o_p, [x.astype(np.float64) for x in g], o_m, o_v, step=1, **hp)
+    torch.cuda.synchronize()
+    assert ns.check_status() == ns.OK
+    for i in range(len(sizes)):
+        for dev, ref in ((ps[i], o_p[i]), (ms[i], o_m[i]), (vs[i], o_v[i])):
+            assert rel(host64(dev), ref) <= TOL, i

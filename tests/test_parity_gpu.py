@@ -200,3 +200,28 @@ def test_null_grad_skips_matrix():
     torch.cuda.synchronize()
     assert torch.equal(ps[1], before[1]) and torch.equal(ms[1], torch.zeros_like(ms[1]))
     assert not torch.equal(ps[0], before[0]) and not torch.equal(ps[2], before[2])
+
+
+@pytest.mark.parametrize("prec,tol", [("bf16", TOL_O_BF16), ("fp32", TOL_O_FP32)], ids=["bf16", "fp32"])
+def test_step_many_matrices_multi_chunk_tables(prec, tol):
+    """600 small matrices: the per-call tables (matrix records, fused-update problems and, in bf16
+    mode, the parameters' TMA views) exceed one 32,000-byte kernel-parameter chunk and are written
+    in several launches. Every matrix is checked, so a chunk written to the wrong place shows."""
+    import newton_schulz_13_b200 as ns
+    rng = np.random.default_rng(31)
+    shapes = [(16 + 8 * (j % 5), 24 + 8 * (j % 7)) for j in range(600)]
+    p0 = [synth.round_to(0.02 * rng.standard_normal(s), "fp32") for s in shapes]
+    g = [synth.round_to(rng.standard_normal(s), "fp32") for s in shapes]
+    ps = [to_dev(x, torch.float32) for x in p0]
+    ms = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes]
+    ns.muon_step(ps, [to_dev(x, torch.float32) for x in g], ms, lr=0.02, mu=0.95, nesterov=True,
+                 weight_decay=0.0, steps=5, coeffs=Q5, eps=1e-7, prec=prec)
+    torch.cuda.synchronize()
+    assert ns.check_status() == ns.OK
+    for j, s in enumerate(shapes):
+        o_p, o_m = p0[j].astype(np.float64).copy(), np.zeros(s)
+        O_ref = oracle.muon_step([o_p], [g[j]], [o_m], lr=0.02, mu=0.95, nesterov=True, weight_decay=0.0,
+                                 rms_mode=0, coeffs=Q5, zero_center=False, eps=1e-7, want_O=True)[0]
+        O_gpu = (p0[j].astype(np.float64) - host64(ps[j])) / np.float64(np.float32(0.02))
+        assert rel(O_gpu, O_ref) <= tol, (j, rel(O_gpu, O_ref))
+        assert rel(host64(ms[j]), o_m) <= TOL_M, j
