@@ -241,11 +241,18 @@ def run_ours(args, world, rank, local):
               steps=len(wl.coeffs), coeffs=wl.coeffs, zero_center=wl.zero_center, eps=wl.eps, prec=args.prec,
               stream=stream)
 
+    # the step as one muon_step call over all matrices, or as one call per group of whole layers
+    per_call = max(1, wl.layer_size) * args.step_group_layers if args.step_group_layers > 0 else wl.count
+    call_groups = [list(range(j, min(wl.count, j + per_call))) for j in range(0, wl.count, per_call)]
+
     def step():
         if args.sharded:
             sharded.sharded_muon_step(params, grads, mom, **hp)
-        else:
+        elif len(call_groups) == 1:
             ns.muon_step(params, grads, mom, **hp)
+        else:
+            for grp in call_groups:
+                ns.muon_step([params[j] for j in grp], [grads[j] for j in grp], [mom[j] for j in grp], **hp)
 
     for _ in range(args.warmup):
         step()
@@ -313,6 +320,7 @@ def run_ours(args, world, rank, local):
                    "weight_decay": wl.weight_decay, "rms_scale": "sqrt(max(1, rows/cols))",
                    "l2": "no flush: inputs (params+grads+momentum, %.0f GB per GPU) are larger than the "
                          "126 MB L2" % (elements * (4 + 4 + 2 * gbytes) / 1e9),
+                   "muon_step_calls_per_step": len(call_groups),
                    "parallelism": ("one weight set split across GPUs by Newton-Schulz FLOPs, updated parameters "
                                    "all-gathered (strong scaling)") if args.sharded else
                                   "independent weight set per GPU (weak scaling, no collective)"},
@@ -558,9 +566,12 @@ def main(argv=None):
     ap.add_argument("--prec", choices=["bf16", "fp32"], default="bf16",
                     help="Newton-Schulz working precision: bf16 operands (default), or fp32 through "
                          "3xTF32 tensor-core products")
+    ap.add_argument("--step-group-layers", type=int, default=0,
+                    help="device-timed step as one muon_step call per group of this many layers "
+                         "(0: one call over all matrices)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--e2e-group-layers", type=int, default=4,
+    ap.add_argument("--e2e-group-layers", type=int, default=1,
                     help="layers per muon_step call in the pipelined end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--library-baseline", action="store_true",

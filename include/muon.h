@@ -205,6 +205,16 @@ MUON_API int muon_check_status(muon_stream_t stream);
 /* Frees the workspace and cached plans of the current device (synchronises the device). */
 MUON_API int muon_release_workspace(void);
 
+/* Tuning: the largest number of elements (summed over consecutive matrices) that muon_step
+ * processes in one wave of launches (prologue, norm and Newton-Schulz products); a larger matrix
+ * is a wave of its own. Waves only split the launch sequence: the results do not depend on the
+ * setting. Smaller launches keep more of one phase's output in L2 for the next phase and, under
+ * the power cap, run at higher clocks (one Llama-8B step: about 460 ms in waves of two layers
+ * against 520-580 ms in one wave), at the cost of more launches. elements = 0 restores the
+ * default, 2^29; negative values are rejected with MUON_ERR_INVALID_ARG. Applies to calls made
+ * after it (a cached plan built with another setting is rebuilt). */
+MUON_API int muon_set_wave_elements(int64_t elements);
+
 /* Kernel classes counted and timed by the library, indices into muon_profile_read's arrays. */
 enum {
   MUON_KC_CENTER = 0,   /* column sums and means for zero-centring                    */

@@ -31,7 +31,7 @@ CUBIC = (1.5, -0.5, 0.0)
 
 EXPORTS = ["muon_ns_orthogonalize", "muon_step", "muon_adamw_step", "muon_last_error",
            "muon_check_status", "muon_release_workspace", "muon_profile_enable", "muon_profile_read",
-           "muon_launch_count", "muon_version"]
+           "muon_launch_count", "muon_version", "muon_set_wave_elements"]
 
 
 class MuonError(RuntimeError):
@@ -45,9 +45,17 @@ class Coeffs(ctypes.Structure):
 
 
 def _load() -> ctypes.CDLL:
+    # the library is built in-tree from csrc/ with nvcc when it is missing or older than its
+    # sources; there is no fallback implementation if that fails
+    from . import build as _build
+    if _build.stale():
+        try:
+            _build.build()
+        except Exception as e:  # noqa: BLE001
+            raise ImportError(f"{LIB_PATH} is missing or out of date and building it failed ({e}); "
+                              "there is no fallback implementation") from e
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m newton_schulz_13_b200.build` "
-                          "(there is no fallback implementation)")
+        raise ImportError(f"{LIB_PATH} is missing (there is no fallback implementation)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, i64p = ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)
     vpp = ctypes.POINTER(ctypes.c_void_p)
@@ -68,6 +76,8 @@ def _load() -> ctypes.CDLL:
     lib.muon_check_status.restype = ctypes.c_int
     lib.muon_check_status.argtypes = [vp]
     lib.muon_release_workspace.restype = ctypes.c_int
+    lib.muon_set_wave_elements.restype = ctypes.c_int
+    lib.muon_set_wave_elements.argtypes = [ctypes.c_int64]
     lib.muon_profile_enable.restype = ctypes.c_int
     lib.muon_profile_enable.argtypes = [ctypes.c_int]
     lib.muon_profile_read.restype = ctypes.c_int
@@ -212,6 +222,12 @@ def check_status(stream=None) -> int:
 
 def release_workspace() -> None:
     _check(lib.muon_release_workspace())
+
+
+def set_wave_elements(elements: int = 0) -> None:
+    """Largest number of elements muon_step processes in one wave of launches (0: the default,
+    2^29). Results do not depend on it; see muon_set_wave_elements in include/muon.h."""
+    _check(lib.muon_set_wave_elements(int(elements)))
 
 
 def profile_enable(on: bool = True) -> None:

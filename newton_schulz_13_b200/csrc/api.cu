@@ -2,7 +2,7 @@
 // (workspace layout, TMA descriptors, grouped problem tables) and the launch sequence.
 //
 // Launch sequence of one muon_step (all on the caller's stream, no host synchronisation once the
-// plan exists):
+// plan exists), once per wave of matrices (see kWaveElements):
 //   [column sums, column means]   only with zero-centring
 //   prologue                      momentum, Nesterov, norm partials, U = cast(u)
 //   norm                          alpha_j = 1 / (||u_j||_F + eps)
@@ -124,15 +124,36 @@ struct BufMapsX3 {   // TMA views of one two-plane fp32 buffer: K-major and MN-m
   int k128 = -1, mn32 = -1;
 };
 
+// Matrices are processed in waves: consecutive runs of matrices of at most kWaveElements elements
+// in total (a larger matrix is a wave of its own). Each wave runs its own prologue, norm and
+// Newton-Schulz launches. Within one launch over a few hundred million elements, the output of
+// one phase (A, B, the new iterate) is partly still in L2 when the next phase reads it; launches
+// over the whole Llama-8B set (7e9 elements) measured 12-25 % slower per step under the power
+// cap (lower SM clock at the same board power), with per-wave launch tails costing about 3 %.
+constexpr int64_t kWaveElements = int64_t(1) << 29;
+int64_t g_wave_elements = kWaveElements;   // muon_set_wave_elements
+
+// A wave: matrices [j0, j1) of the plan. Every prefix sum in the device tables (elementwise
+// chunks, column-sum items, product tiles) restarts at zero at the wave's first matrix, so a
+// wave's launches take the table sub-ranges starting at j0 and need no offsets.
+struct Wave {
+  int j0 = 0, j1 = 0;
+  int64_t n_chunks = 0, cs_items = 0, cm_items = 0;
+  uint32_t tiles_gram = 0, tiles_poly = 0, tiles_upd = 0;
+  double fl_gram = 0, fl_poly = 0, fl_upd = 0;      // nominal flops per launch
+  double ex_gram = 0, ex_poly = 0, ex_upd = 0;      // executed (tile) flops per launch
+};
+
 struct Plan {
   std::vector<Shape> shapes;
   int x_bf16 = 1;
+  int64_t wave_elements = 0;
   char* ws = nullptr;
   size_t ws_bytes = 0;
   // device tables
   MatInfo* d_mats = nullptr;
   float* d_partials = nullptr;
-  int64_t n_chunks = 0, cs_items = 0, cm_items = 0;
+  std::vector<Wave> waves;
   // per-matrix workspace pointers
   std::vector<void*> x0, x1, A, B;
   std::vector<float*> colmean, colpart, alpha;
@@ -142,9 +163,6 @@ struct Plan {
   void* d_poly = nullptr;
   void* d_updB[2] = {nullptr, nullptr};
   void* d_updA[2] = {nullptr, nullptr};
-  uint32_t tiles_gram = 0, tiles_poly = 0, tiles_upd = 0;
-  double fl_gram = 0, fl_poly = 0, fl_upd = 0;      // nominal flops per launch
-  double ex_gram = 0, ex_poly = 0, ex_upd = 0;      // executed (tile) flops per launch
   // per-call MatInfo table (written through kernel parameters when it changes)
   std::vector<MatInfo> last_uploaded;
   bool uploaded_once = false;
@@ -211,7 +229,8 @@ int device_state(DeviceState** out) {
 
 // Builds the workspace, TMA descriptors and grouped problem tables for a list of shapes.
 int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Plan** out) {
-  if (ds.plan && ds.plan->shapes == shapes && ds.plan->x_bf16 == x_bf16) {
+  if (ds.plan && ds.plan->shapes == shapes && ds.plan->x_bf16 == x_bf16 &&
+      ds.plan->wave_elements == g_wave_elements) {
     *out = ds.plan.get();
     return MUON_OK;
   }
@@ -219,19 +238,45 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   std::unique_ptr<Plan> P(new Plan());
   P->shapes = shapes;
   P->x_bf16 = x_bf16;
+  P->wave_elements = g_wave_elements;
   const int n = (int)shapes.size();
   // bf16 mode: one bf16 plane per buffer; fp32 mode: hi and lo fp32 planes (GemmProblemX3)
   const size_t esz = x_bf16 ? 2 : 8;
   const size_t AL = 256;
 
+  // ---- waves
+  std::vector<int> wave_of(n);
+  {
+    int64_t acc = 0;
+    for (int j = 0; j < n; ++j) {
+      const int64_t el = shapes[j].r * shapes[j].c;
+      if (j == 0 || acc + el > P->wave_elements) {
+        P->waves.emplace_back();
+        P->waves.back().j0 = j;
+        acc = 0;
+      }
+      acc += el;
+      P->waves.back().j1 = j + 1;
+      wave_of[j] = (int)P->waves.size() - 1;
+    }
+  }
+  auto wave_start = [&](int j) { return P->waves[wave_of[j]].j0 == j; };
+
   // ---- layout
-  size_t off = 0;
+  // The per-matrix buffers (X0, X1, A, B, column-mean scratch) of one wave are laid out from the
+  // start of the workspace; the next wave reuses the same region, since waves run one after the
+  // other in stream order. The region is as large as the largest wave.
+  size_t off = 0, wave_region = 0;
   std::vector<size_t> o_x0(n), o_x1(n), o_A(n), o_B(n), o_cm(n), o_cp(n);
   P->ldx.resize(n);
   P->ldm.resize(n);
-  int64_t chunks = 0, cs = 0, cm = 0;
+  int64_t chunks = 0, cs = 0, cm = 0, max_chunks = 0;
   std::vector<MatInfo> mats(n);
   for (int j = 0; j < n; ++j) {
+    if (wave_start(j)) {
+      chunks = cs = cm = 0;
+      off = 0;
+    }
     const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c);
     const int64_t ldx = align_up(c, 8), ldm = align_up(m, 8);
     P->ldx[j] = ldx;
@@ -243,6 +288,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     o_cm[j] = off; off = align_up(off + (size_t)c * 4, AL);
     const int64_t n_rc = ceil_div(r, kCsRows), n_cb = ceil_div(c, kCsCols);
     o_cp[j] = off; off = align_up(off + (size_t)n_rc * c * 4, AL);
+    wave_region = std::max(wave_region, off);
     MatInfo& mi = mats[j];
     std::memset(&mi, 0, sizeof(mi));
     mi.rows = r; mi.cols = c; mi.ldx = ldx;
@@ -250,9 +296,15 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     mi.chunk_begin = chunks; chunks += ceil_div(r * c, kChunk);
     mi.cs_begin = cs; cs += n_rc * n_cb;
     mi.cm_begin = cm; cm += n_cb;
+    Wave& w = P->waves[wave_of[j]];
+    w.n_chunks = chunks;
+    w.cs_items = cs;
+    w.cm_items = cm;
+    max_chunks = std::max(max_chunks, chunks);
   }
+  off = wave_region;
   const size_t o_alpha = off; off = align_up(off + (size_t)n * 4, AL);
-  const size_t o_part = off; off = align_up(off + (size_t)chunks * 4, AL);
+  const size_t o_part = off; off = align_up(off + (size_t)max_chunks * 4, AL);
   const size_t o_mats = off; off = align_up(off + (size_t)n * sizeof(MatInfo), AL);
   const int maps_per = x_bf16 ? 12 : 8;   // 4 buffers x 3 views (bf16) or x 2 views (fp32)
   const size_t o_maps = off;
@@ -275,9 +327,6 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     return fail(MUON_ERR_WORKSPACE, buf);
   }
   char* W = P->ws;
-  P->n_chunks = chunks;
-  P->cs_items = cs;
-  P->cm_items = cm;
   P->d_partials = reinterpret_cast<float*>(W + o_part);
   P->d_mats = reinterpret_cast<MatInfo*>(W + o_mats);
   for (int j = 0; j < n; ++j) {
@@ -329,6 +378,8 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     std::vector<GemmProblem> gram[2], poly, updB[2], updA[2];
     uint32_t tg = 0, tp = 0, tu = 0;
     for (int j = 0; j < n; ++j) {
+      if (wave_start(j)) tg = tp = tu = 0;
+      Wave& w = P->waves[wave_of[j]];
       const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c), nn = std::max(r, c);
       const bool tall = r > c;
       BufMaps mx[2] = {make3(j, 0, P->x0[j], r, c, P->ldx[j]), make3(j, 1, P->x1[j], r, c, P->ldx[j])};
@@ -390,16 +441,16 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       tg += gram[0].back().n_tiles;
       tp += q.n_tiles;
       tu += updB[0].back().n_tiles;
-      P->fl_gram += 2.0 * m * m * nn;
-      P->fl_poly += 2.0 * m * m * m;
-      P->fl_upd += 2.0 * m * m * nn;
+      w.tiles_gram = tg; w.tiles_poly = tp; w.tiles_upd = tu;
+      w.fl_gram += 2.0 * m * m * nn;
+      w.fl_poly += 2.0 * m * m * m;
+      w.fl_upd += 2.0 * m * m * nn;
       const double tile_fl = 2.0 * kTcPairBM * kTcBN;
-      P->ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kTcBK) * kTcBK);
-      P->ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
-      P->ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
+      w.ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kTcBK) * kTcBK);
+      w.ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
+      w.ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
     }
     if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
-    P->tiles_gram = tg; P->tiles_poly = tp; P->tiles_upd = tu;
     MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
     std::vector<GemmProblem>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
@@ -444,6 +495,8 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     std::vector<GemmProblemX3> gram[2], poly, updB[2], updA[2];
     uint32_t tg = 0, tp = 0, tu = 0;
     for (int j = 0; j < n; ++j) {
+      if (wave_start(j)) tg = tp = tu = 0;
+      Wave& w = P->waves[wave_of[j]];
       const int64_t r = shapes[j].r, c = shapes[j].c, m = std::min(r, c), nn = std::max(r, c);
       const bool tall = r > c;
       const int64_t ldx = P->ldx[j], ldm = P->ldm[j];
@@ -501,17 +554,17 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       tg += gram[0].back().n_tiles;
       tp += q.n_tiles;
       tu += updB[0].back().n_tiles;
-      P->fl_gram += 2.0 * m * m * nn;
-      P->fl_poly += 2.0 * m * m * m;
-      P->fl_upd += 2.0 * m * m * nn;
+      w.tiles_gram = tg; w.tiles_poly = tp; w.tiles_upd = tu;
+      w.fl_gram += 2.0 * m * m * nn;
+      w.fl_poly += 2.0 * m * m * m;
+      w.fl_upd += 2.0 * m * m * nn;
       // executed: three tf32 products per tile and K step
       const double tile_fl = 3.0 * 2.0 * kTcPairBM * kTcBN;
-      P->ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kX3BK) * kX3BK);
-      P->ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kX3BK) * kX3BK);
-      P->ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kX3BK) * kX3BK);
+      w.ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kX3BK) * kX3BK);
+      w.ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kX3BK) * kX3BK);
+      w.ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kX3BK) * kX3BK);
     }
     if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
-    P->tiles_gram = tg; P->tiles_poly = tp; P->tiles_upd = tu;
     MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
     std::vector<GemmProblemX3>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
@@ -643,10 +696,14 @@ int check_shape(int64_t r, int64_t c, const char* what) {
   return MUON_OK;
 }
 
-// Runs the Newton-Schulz phases for every matrix of the plan.
-int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaStream_t s,
+// Runs the Newton-Schulz phases for the matrices of one wave. fused_last (optional) is the
+// per-call table of last-update problems for all matrices of the plan.
+int run_ns(DeviceState& ds, Plan& P, const Wave& w, const std::vector<muon_coeffs_t>& co, cudaStream_t s,
            const void* fused_last = nullptr, float lr = 0.0f, float decay = 1.0f) {
-  const int n = (int)P.shapes.size();
+  const int n = w.j1 - w.j0;
+  // the wave's sub-range of a problem table
+  auto tc = [&](void* t) { return static_cast<GemmProblem*>(t) + w.j0; };
+  auto x3 = [&](void* t) { return static_cast<GemmProblemX3*>(t) + w.j0; };
   for (size_t k = 0; k < co.size(); ++k) {
     const int p = (int)(k & 1);
     const int first = k == 0 ? 1 : 0;
@@ -660,12 +717,12 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
     EpiScalars eg{1.0f, 0.0f, first ? 2 : 0, 0, 0.0f};
     if (P.x_bf16 && c.c == 0.0f) eg = EpiScalars{c.b, 0.0f, first ? 2 : 0, 0, c.a};
     if (P.x_bf16) {
-      e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
-        return launch_gemm_tc_pair(static_cast<GemmProblem*>(P.d_gram[p]), n, P.tiles_gram, eg, ds.d_status, ds.pair_capacity, s);
+      e = timed_launch(MUON_KC_GEMM, s, w.fl_gram, w.ex_gram, [&] {
+        return launch_gemm_tc_pair(tc(P.d_gram[p]), n, w.tiles_gram, eg, ds.d_status, ds.pair_capacity, s);
       }, MUON_KC_GEMM_GRAM);
     } else {
-      e = timed_launch(MUON_KC_GEMM, s, P.fl_gram, P.ex_gram, [&] {
-        return launch_gemm_x3(static_cast<GemmProblemX3*>(P.d_gram[p]), n, P.tiles_gram, eg, ds.d_status, ds.x3_capacity, s);
+      e = timed_launch(MUON_KC_GEMM, s, w.fl_gram, w.ex_gram, [&] {
+        return launch_gemm_x3(x3(P.d_gram[p]), n, w.tiles_gram, eg, ds.d_status, ds.x3_capacity, s);
       }, MUON_KC_GEMM_GRAM);
     }
     if (e != cudaSuccess) return cuda_fail(e, "gram launch");
@@ -674,12 +731,12 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
     if (c.c != 0.0f) {
       EpiScalars ep{c.c, c.b, 0, 0, P.x_bf16 ? c.a : 0.0f};
       if (P.x_bf16) {
-        e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
-          return launch_gemm_tc_pair(static_cast<GemmProblem*>(P.d_poly), n, P.tiles_poly, ep, ds.d_status, ds.pair_capacity, s);
+        e = timed_launch(MUON_KC_GEMM, s, w.fl_poly, w.ex_poly, [&] {
+          return launch_gemm_tc_pair(tc(P.d_poly), n, w.tiles_poly, ep, ds.d_status, ds.pair_capacity, s);
         }, MUON_KC_GEMM_POLY);
       } else {
-        e = timed_launch(MUON_KC_GEMM, s, P.fl_poly, P.ex_poly, [&] {
-          return launch_gemm_x3(static_cast<GemmProblemX3*>(P.d_poly), n, P.tiles_poly, ep, ds.d_status, ds.x3_capacity, s);
+        e = timed_launch(MUON_KC_GEMM, s, w.fl_poly, w.ex_poly, [&] {
+          return launch_gemm_x3(x3(P.d_poly), n, w.tiles_poly, ep, ds.d_status, ds.x3_capacity, s);
         }, MUON_KC_GEMM_POLY);
       }
       if (e != cudaSuccess) return cuda_fail(e, "poly launch");
@@ -696,12 +753,12 @@ int run_ns(DeviceState& ds, Plan& P, const std::vector<muon_coeffs_t>& co, cudaS
       eu.fused = 1;
     }
     if (P.x_bf16) {
-      e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
-        return launch_gemm_tc_pair(static_cast<GemmProblem*>(upd), n, P.tiles_upd, eu, ds.d_status, ds.pair_capacity, s);
+      e = timed_launch(MUON_KC_GEMM, s, w.fl_upd, w.ex_upd, [&] {
+        return launch_gemm_tc_pair(tc(upd), n, w.tiles_upd, eu, ds.d_status, ds.pair_capacity, s);
       }, MUON_KC_GEMM_UPDATE);
     } else {
-      e = timed_launch(MUON_KC_GEMM, s, P.fl_upd, P.ex_upd, [&] {
-        return launch_gemm_x3(static_cast<GemmProblemX3*>(upd), n, P.tiles_upd, eu, ds.d_status, ds.x3_capacity, s);
+      e = timed_launch(MUON_KC_GEMM, s, w.fl_upd, w.ex_upd, [&] {
+        return launch_gemm_x3(x3(upd), n, w.tiles_upd, eu, ds.d_status, ds.x3_capacity, s);
       }, MUON_KC_GEMM_UPDATE);
     }
     if (e != cudaSuccess) return cuda_fail(e, "update launch");
@@ -807,6 +864,14 @@ int muon_release_workspace(void) {
   return MUON_OK;
 }
 
+int muon_set_wave_elements(int64_t elements) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  t_err.clear();
+  if (elements < 0) return fail(MUON_ERR_INVALID_ARG, "elements must be >= 0");
+  g_wave_elements = elements == 0 ? kWaveElements : elements;
+  return MUON_OK;
+}
+
 int muon_step(int count, float* const* params, const void* const* grads, muon_dtype_t grad_dtype,
               float* const* momentum, const int64_t* rows, const int64_t* cols, float lr, float mu,
               int nesterov, float weight_decay, muon_rms_t rms_scale, int steps,
@@ -884,28 +949,32 @@ int muon_step(int count, float* const* params, const void* const* grads, muon_dt
   }
 
   const int ew_grid = ds->sms * 8;
-  cudaError_t e;
-  if (zero_center) {
-    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colsum(P->d_mats, n, P->cs_items, g_bf16, s); });
-    if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
-    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colmean(P->d_mats, n, P->cm_items, s); });
-    if (e != cudaSuccess) return cuda_fail(e, "column-mean launch");
+  for (const Wave& w : P->waves) {
+    const MatInfo* dm = P->d_mats + w.j0;
+    const int nw = w.j1 - w.j0;
+    cudaError_t e;
+    if (zero_center) {
+      e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colsum(dm, nw, w.cs_items, g_bf16, s); });
+      if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
+      e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colmean(dm, nw, w.cm_items, s); });
+      if (e != cudaSuccess) return cuda_fail(e, "column-mean launch");
+    }
+    e = timed_launch(MUON_KC_PROLOGUE, s, 0, 0, [&] {
+      return launch_prologue(dm, nw, w.n_chunks, g_bf16, x_bf16, 1, mu, nesterov, zero_center,
+                             P->d_partials, ds->d_status, ew_grid, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+    e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(dm, nw, P->d_partials, eps, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "norm launch");
+    rc = run_ns(*ds, *P, w, co, s, fused, lr, 1.0f - lr * weight_decay);
+    if (rc != MUON_OK) return rc;
+    if (fused) continue;   // the last update product already wrote the parameters
+    e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
+      return launch_update(dm, nw, w.n_chunks, x_bf16, lr, 1.0f - lr * weight_decay, steps == 0 ? 1 : 0,
+                           ew_grid, s);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
   }
-  e = timed_launch(MUON_KC_PROLOGUE, s, 0, 0, [&] {
-    return launch_prologue(P->d_mats, n, P->n_chunks, g_bf16, x_bf16, 1, mu, nesterov, zero_center,
-                           P->d_partials, ds->d_status, ew_grid, s);
-  });
-  if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
-  e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(P->d_mats, n, P->d_partials, eps, s); });
-  if (e != cudaSuccess) return cuda_fail(e, "norm launch");
-  rc = run_ns(*ds, *P, co, s, fused, lr, 1.0f - lr * weight_decay);
-  if (rc != MUON_OK) return rc;
-  if (fused) return MUON_OK;   // the last update GEMM already wrote the parameters
-  e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
-    return launch_update(P->d_mats, n, P->n_chunks, x_bf16, lr, 1.0f - lr * weight_decay, steps == 0 ? 1 : 0,
-                         ew_grid, s);
-  });
-  if (e != cudaSuccess) return cuda_fail(e, "epilogue launch");
   return MUON_OK;
 }
 
@@ -1032,24 +1101,25 @@ int muon_ns_orthogonalize(const void* G, muon_dtype_t g_dtype, void* X, muon_dty
   if (rc != MUON_OK) return rc;
   const int g_bf16 = g_dtype == MUON_BF16;
   const int ew_grid = ds->sms * 8;
+  const Wave& w = P->waves[0];   // one matrix: one wave
   cudaError_t e;
   if (zero_center) {
-    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colsum(P->d_mats, 1, P->cs_items, g_bf16, s); });
+    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colsum(P->d_mats, 1, w.cs_items, g_bf16, s); });
     if (e != cudaSuccess) return cuda_fail(e, "column-sum launch");
-    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colmean(P->d_mats, 1, P->cm_items, s); });
+    e = timed_launch(MUON_KC_CENTER, s, 0, 0, [&] { return launch_colmean(P->d_mats, 1, w.cm_items, s); });
     if (e != cudaSuccess) return cuda_fail(e, "column-mean launch");
   }
   e = timed_launch(MUON_KC_PROLOGUE, s, 0, 0, [&] {
-    return launch_prologue(P->d_mats, 1, P->n_chunks, g_bf16, x_bf16, 0, 0.0f, 0, zero_center,
+    return launch_prologue(P->d_mats, 1, w.n_chunks, g_bf16, x_bf16, 0, 0.0f, 0, zero_center,
                            P->d_partials, ds->d_status, ew_grid, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
   e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(P->d_mats, 1, P->d_partials, eps, s); });
   if (e != cudaSuccess) return cuda_fail(e, "norm launch");
-  rc = run_ns(*ds, *P, co, s);
+  rc = run_ns(*ds, *P, w, co, s);
   if (rc != MUON_OK) return rc;
   e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
-    return launch_output(P->d_mats, 1, P->n_chunks, x_bf16, x_dtype == MUON_BF16, steps == 0 ? 1 : 0,
+    return launch_output(P->d_mats, 1, w.n_chunks, x_bf16, x_dtype == MUON_BF16, steps == 0 ? 1 : 0,
                          ew_grid, s);
   });
   if (e != cudaSuccess) return cuda_fail(e, "output launch");

@@ -169,3 +169,11 @@ def test_adamw_no_device_fails_loudly():
     import newton_schulz_13_b200 as ns
     assert _adam(ns) == ns.ERR_UNSUPPORTED
     assert _adam(ns, numel=[0]) == ns.OK   # nothing to do: no device needed
+
+
+def test_set_wave_elements_rejects_negative_values():
+    import newton_schulz_13_b200 as ns
+    with pytest.raises(ns.MuonError):
+        ns.set_wave_elements(-1)
+    ns.set_wave_elements(1 << 20)
+    ns.set_wave_elements(0)

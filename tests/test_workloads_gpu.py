@@ -185,3 +185,40 @@ def test_llama8b_full_size():
         want = np.sqrt(np.sum(scalar_map(np.sqrt(np.clip(sig2, 0, None)), wl.coeffs) ** 2))
         got = np.linalg.norm(O)
         assert abs(got / want - 1.0) <= 0.02, (j, "frobenius", got, want)
+
+
+# ----------------------------------------------------------------------------- waves
+@pytest.fixture
+def small_waves():
+    import newton_schulz_13_b200 as ns
+    yield ns.set_wave_elements
+    ns.set_wave_elements(0)
+
+
+@pytest.mark.parametrize("name,prec,wave", [("gpt2_small", "bf16", 1 << 22), ("gpt2_small", "fp32", 1 << 22),
+                                            ("cubic_zero_center_12", "bf16", 1 << 20),
+                                            ("mamba_24", "bf16", 1 << 21)])
+def test_waves_give_identical_results(small_waves, name, prec, wave):
+    """Splitting a call into waves of launches changes no arithmetic: the parameters and momentum
+    after two steps are bit-identical to those of the one-wave run (tiny waves: 20-100 of them)."""
+    wl = synth.WORKLOADS[name]
+    outs = []
+    for w in (0, wave):
+        small_waves(w)
+        case = StepCase(wl, sample=[], device_fill=True)
+        for k in range(2):
+            case.step(k, prec=prec)
+        torch.cuda.synchronize()
+        outs.append([p.clone() for p in case.params] + [m.clone() for m in case.momentum])
+    import newton_schulz_13_b200 as ns
+    assert ns.check_status() == ns.OK
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_waves_against_the_oracle(small_waves):
+    """Many waves on GPT-2-small (about three matrices each), checked against the fp64 oracle on
+    matrices in the first, a middle and the last wave."""
+    small_waves(1 << 22)
+    wl = synth.WORKLOADS["gpt2_small"]
+    run_and_check(StepCase(wl, sample=[0, 21, 46, 47], device_fill=True), 2)
