@@ -215,6 +215,7 @@ def run_ours(args, world, rank, local):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    ns.set_wave_elements(args.wave_elements)
     if world > 1:
         import torch.distributed as dist
         import datetime
@@ -321,6 +322,7 @@ def run_ours(args, world, rank, local):
                    "l2": "no flush: inputs (params+grads+momentum, %.0f GB per GPU) are larger than the "
                          "126 MB L2" % (elements * (4 + 4 + 2 * gbytes) / 1e9),
                    "muon_step_calls_per_step": len(call_groups),
+                   "wave_elements": args.wave_elements or (1 << 29),
                    "parallelism": ("one weight set split across GPUs by Newton-Schulz FLOPs, updated parameters "
                                    "all-gathered (strong scaling)") if args.sharded else
                                   "independent weight set per GPU (weak scaling, no collective)"},
@@ -566,6 +568,8 @@ def main(argv=None):
     ap.add_argument("--prec", choices=["bf16", "fp32"], default="bf16",
                     help="Newton-Schulz working precision: bf16 operands (default), or fp32 through "
                          "3xTF32 tensor-core products")
+    ap.add_argument("--wave-elements", type=int, default=0,
+                    help="muon_step wave budget in elements (0: the library default, 2^29)")
     ap.add_argument("--step-group-layers", type=int, default=0,
                     help="device-timed step as one muon_step call per group of this many layers "
                          "(0: one call over all matrices)")
