@@ -20,16 +20,22 @@
  *                                               "Muon meets Mamba" section 4.2)
  *
  * All arithmetic runs in hand-written sm_100a kernels: a fused elementwise prologue, the
- * Newton-Schulz matrix products on the tcgen05 tensor cores (bf16 operands, fp32
- * accumulation in tensor memory), and a fused elementwise epilogue. There is no CPU fallback:
- * on a machine without an sm_100 device every compute call fails with MUON_ERR_UNSUPPORTED.
+ * Newton-Schulz matrix products on the tcgen05 tensor cores (bf16 operands with fp32
+ * accumulation in tensor memory, or fp32 accuracy through 3xTF32 products), with the parameter
+ * update fused into the last product. There is no CPU fallback: on a machine without an sm_100
+ * device every compute call fails with MUON_ERR_UNSUPPORTED.
  *
  * Conventions shared by every call:
  *   - Matrices are dense, row-major, contiguous (leading dimension = cols).
  *   - Pointers named "device" must be device memory (or managed memory) of the current device.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream) and
- *     never synchronise the host, except the first call with a new set of shapes, which
- *     allocates the library's workspace (cudaMalloc) and uploads its tables.
+ *     never synchronise the host, except the first call with a new set of shapes (or precision,
+ *     or wave budget), which allocates the library's workspace (cudaMalloc) and uploads its
+ *     tables. Per-call tables (the caller's pointers) travel to the device inside kernel launch
+ *     parameters, so they never wait behind the caller's own copies on a copy engine.
+ *   - muon_step processes its matrices in waves of consecutive matrices (see
+ *     muon_set_wave_elements); the workspace holds one wave's buffers, about 4 bytes per element
+ *     of the largest wave in bf16 working precision and 16 in fp32.
  *   - The workspace is owned by the library, per process, and shared by all calls: calls must be
  *     ordered (same stream, or synchronised by the caller). Concurrent calls race.
  *   - Argument errors are detected before any device work is enqueued; the call then returns a
@@ -128,9 +134,10 @@ MUON_API int muon_ns_orthogonalize(const void* G, muon_dtype_t g_dtype, void* X,
  *   rms_scale   the RMS factor s (muon_rms_t).
  *   steps, coeffs, zero_center, eps, prec   as for muon_ns_orthogonalize.
  * params[i] and momentum[i] must not overlap each other or any other matrix's buffers.
- * All `count` matrices are processed by the same kernel launches (one prologue, one grouped
- * tensor-core launch per Newton-Schulz phase, one epilogue), so small matrices are not
- * launch-bound. Returns MUON_OK or a negative error code.
+ * The matrices of one wave (consecutive matrices of at most 2^29 elements in total, see
+ * muon_set_wave_elements) share the same kernel launches (one prologue, one norm, one grouped
+ * tensor-core launch per Newton-Schulz phase, the last of which also updates the parameters),
+ * so small matrices are not launch-bound. Returns MUON_OK or a negative error code.
  */
 MUON_API int muon_step(int count, float* const* params, const void* const* grads, muon_dtype_t grad_dtype,
               float* const* momentum, const int64_t* rows, const int64_t* cols, float lr, float mu,
