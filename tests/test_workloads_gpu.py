@@ -187,6 +187,28 @@ def test_llama8b_full_size():
         assert abs(got / want - 1.0) <= 0.02, (j, "frobenius", got, want)
 
 
+def test_llama8b_full_size_fp32_mode():
+    """The whole Llama-8B set in fp32 working precision (3xTF32 products, 14 waves sharing one
+    9.8 GB workspace region), checked against the oracle on the matrices it finishes in seconds:
+    Wk and Wv of layer 0 (first wave) and Wk of layer 31 (last wave)."""
+    import newton_schulz_13_b200 as ns
+    wl = synth.WORKLOADS["llama8b"]
+    exact = [1, 2, 218]
+    case = StepCase(wl, sample=exact, device_fill=True)
+    p_prev = {j: host64(case.params[j]) for j in exact}
+    _, O_ref = case.step(0, prec="fp32")
+    torch.cuda.synchronize()
+    assert ns.check_status() == ns.OK
+    decay = np.float64(np.float32(1.0 - np.float32(wl.lr) * np.float32(wl.weight_decay)))
+    lr32 = np.float64(np.float32(wl.lr))
+    for j in exact:
+        p_new = host64(case.params[j])
+        O_gpu = (p_prev[j] * decay - p_new) / (lr32 * case.rms(j))
+        assert rel(O_gpu, O_ref[j]) <= TOL_O_FP32, (j, rel(O_gpu, O_ref[j]))
+        assert rel(p_new, case.o_params[j]) <= TOL_P, j
+        assert rel(host64(case.momentum[j]), case.o_mom[j]) <= TOL_M, j
+
+
 # ----------------------------------------------------------------------------- waves
 @pytest.fixture
 def small_waves():
