@@ -138,6 +138,7 @@ int64_t g_wave_elements = kWaveElements;   // muon_set_wave_elements
 // wave's launches take the table sub-ranges starting at j0 and need no offsets.
 struct Wave {
   int j0 = 0, j1 = 0;
+  bool wide = false;   // bf16 Gram and update products on 256 x 512 tiles (see build_plan)
   int64_t n_chunks = 0, cs_items = 0, cm_items = 0;
   uint32_t tiles_gram = 0, tiles_poly = 0, tiles_upd = 0;
   double fl_gram = 0, fl_poly = 0, fl_upd = 0;      // nominal flops per launch
@@ -261,6 +262,21 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     }
   }
   auto wave_start = [&](int j) { return P->waves[wave_of[j]].j0 == j; };
+  // Tile width of a wave's Gram and update products (bf16). The 256 x 512 tile reads a quarter
+  // fewer operand bytes per FLOP, which pays for large matrices (Llama-8B step 15 % faster), but on
+  // small ones its column padding and the halved tile count (load balance over the CTA pairs)
+  // cost more (GPT-2-small and Mamba steps 25 % slower). Wide tiles are used when matrices with
+  // min(rows, cols) >= 2048 carry at least 80 % of the wave's Newton-Schulz FLOPs.
+  for (Wave& w : P->waves) {
+    double big = 0.0, all = 0.0;
+    for (int j = w.j0; j < w.j1; ++j) {
+      const double m = (double)std::min(shapes[j].r, shapes[j].c), nn = (double)std::max(shapes[j].r, shapes[j].c);
+      const double f = m * m * nn;
+      all += f;
+      if (m >= 2048) big += f;
+    }
+    w.wide = all > 0.0 && big >= 0.8 * all;
+  }
 
   // ---- layout
   // The per-matrix buffers (X0, X1, A, B, column-mean scratch) of one wave are laid out from the
@@ -346,6 +362,13 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     const int64_t t = ceil_div(m, kTcPairBM);
     return t * (t + 1) / 2;
   };
+  // the same on wide tiles (256 x 512): row block bi starts at column block (256 bi) / 512
+  auto sym_tiles_wide = [](int64_t m) {
+    const int64_t tm = ceil_div(m, kTcPairBM), tn = ceil_div(m, kTcWideBN);
+    int64_t t = 0;
+    for (int64_t bi = 0; bi < tm; ++bi) t += tn - (bi * kTcPairBM) / kTcWideBN;
+    return t;
+  };
   if (x_bf16) {
     PFN_encodeTiled_t encode = get_encode();
     if (!encode) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
@@ -398,9 +421,9 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
         g.M = g.N = (uint32_t)m;
         g.K = (uint32_t)nn;
         g.tiles_m = (uint32_t)ceil_div(m, kTcPairBM);
-        g.tiles_n = (uint32_t)ceil_div(m, kTcBN);
+        g.tiles_n = (uint32_t)ceil_div(m, w.wide ? kTcWideBN : kTcBN);
         g.sym = 1;
-        g.n_tiles = (uint32_t)sym_tiles(m);
+        g.n_tiles = (uint32_t)(w.wide ? sym_tiles_wide(m) : sym_tiles(m));
         g.tile_begin = tg;
         gram[p].push_back(g);
         for (int which = 0; which < 2; ++which) {   // 0: operand B, 1: operand A
@@ -419,7 +442,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
           u.alpha = P->alpha[j];
           u.M = (uint32_t)r; u.N = (uint32_t)c; u.K = (uint32_t)m;
           u.tiles_m = (uint32_t)ceil_div(r, kTcPairBM);
-          u.tiles_n = (uint32_t)ceil_div(c, kTcBN);
+          u.tiles_n = (uint32_t)ceil_div(c, w.wide ? kTcWideBN : kTcBN);
           u.n_tiles = u.tiles_m * u.tiles_n;
           u.tile_begin = tu;
           (which == 0 ? updB[p] : updA[p]).push_back(u);
@@ -433,6 +456,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       q.tma_c = M_(mA.st32);
       q.alpha = P->alpha[j];
       q.M = q.N = q.K = (uint32_t)m;
+      // the polynomial product (K = m) stays on 256 x 256 tiles: its triangle wastes less there
       q.tiles_m = (uint32_t)ceil_div(m, kTcPairBM); q.tiles_n = (uint32_t)ceil_div(m, kTcBN);
       q.sym = 1;
       q.n_tiles = (uint32_t)sym_tiles(m);
@@ -445,10 +469,10 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       w.fl_gram += 2.0 * m * m * nn;
       w.fl_poly += 2.0 * m * m * m;
       w.fl_upd += 2.0 * m * m * nn;
-      const double tile_fl = 2.0 * kTcPairBM * kTcBN;
-      w.ex_gram += tile_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kTcBK) * kTcBK);
+      const double tile_fl = 2.0 * kTcPairBM * kTcBN, gu_fl = 2.0 * kTcPairBM * (w.wide ? kTcWideBN : kTcBN);
+      w.ex_gram += gu_fl * gram[0].back().n_tiles * (double)(ceil_div(nn, kTcBK) * kTcBK);
       w.ex_poly += tile_fl * q.n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
-      w.ex_upd += tile_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
+      w.ex_upd += gu_fl * updB[0].back().n_tiles * (double)(ceil_div(m, kTcBK) * kTcBK);
     }
     if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
     MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
@@ -718,7 +742,8 @@ int run_ns(DeviceState& ds, Plan& P, const Wave& w, const std::vector<muon_coeff
     if (P.x_bf16 && c.c == 0.0f) eg = EpiScalars{c.b, 0.0f, first ? 2 : 0, 0, c.a};
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, w.fl_gram, w.ex_gram, [&] {
-        return launch_gemm_tc_pair(tc(P.d_gram[p]), n, w.tiles_gram, eg, ds.d_status, ds.pair_capacity, s);
+        return (w.wide ? launch_gemm_tc_pair_wide : launch_gemm_tc_pair)(tc(P.d_gram[p]), n, w.tiles_gram, eg,
+                                                                         ds.d_status, ds.pair_capacity, s);
       }, MUON_KC_GEMM_GRAM);
     } else {
       e = timed_launch(MUON_KC_GEMM, s, w.fl_gram, w.ex_gram, [&] {
@@ -754,7 +779,8 @@ int run_ns(DeviceState& ds, Plan& P, const Wave& w, const std::vector<muon_coeff
     }
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, w.fl_upd, w.ex_upd, [&] {
-        return launch_gemm_tc_pair(tc(upd), n, w.tiles_upd, eu, ds.d_status, ds.pair_capacity, s);
+        return (w.wide ? launch_gemm_tc_pair_wide : launch_gemm_tc_pair)(tc(upd), n, w.tiles_upd, eu, ds.d_status,
+                                                                         ds.pair_capacity, s);
       }, MUON_KC_GEMM_UPDATE);
     } else {
       e = timed_launch(MUON_KC_GEMM, s, w.fl_upd, w.ex_upd, [&] {

@@ -152,6 +152,9 @@ cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_
                            EpiScalars ep, int* status, int grid, cudaStream_t s);
 cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                 EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
+// The same with 256 x kTcWideBN tiles (problem tables built with tiles_n = ceil(N / kTcWideBN)).
+cudaError_t launch_gemm_tc_pair_wide(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
+                                     EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
 int gemm_tc_pair_capacity(int sms);
 cudaError_t launch_gemm_x3(const GemmProblemX3* probs, int nprobs, uint32_t total_tiles,
                            EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
@@ -163,6 +166,7 @@ constexpr int kTcBM = 128;
 constexpr int kTcPairBM = 256;
 constexpr int kTcBN = 256;
 constexpr int kTcBK = 64;
+constexpr int kTcWideBN = 512;   // CTA-pair wide tiles: kTcPairBM x kTcWideBN (Gram and update products)
 // 3xTF32 kernel: CTA-pair tiles kTcPairBM x kTcBN, K advances kX3BK (one 128-byte row of fp32)
 // per pipeline stage.
 constexpr int kX3BK = 32;

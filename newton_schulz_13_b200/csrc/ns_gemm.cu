@@ -36,21 +36,30 @@ constexpr uint32_t kBoxBytes = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64
 constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-// Geometry of the two variants. Each CTA owns 128 accumulator rows x 256 columns (two
-// accumulators = all 512 tensor-memory columns).
-//   single CTA: output tile 128 x 256, the CTA loads 128 rows of opA and 256 rows of opB.
-//   CTA pair:   output tile 256 x 256; each CTA loads its 128 rows of opA and 128 of the 256 opB
-//               rows, the even CTA issues 256 x 256 x 16 MMAs that read both CTAs' stages.
-template <bool PAIR>
+// Geometry of the variants. Each CTA owns 128 accumulator rows; tensor memory holds 512 columns.
+//   single CTA:  output tile 128 x 256, the CTA loads 128 rows of opA and 256 rows of opB; two
+//                accumulators of 256 columns (the epilogue of one tile overlaps the next tile).
+//   CTA pair:    output tile 256 x 256; each CTA loads its 128 rows of opA and 128 of the 256 opB
+//                rows, the even CTA issues 256 x 256 x 16 MMAs that read both CTAs' stages; two
+//                accumulators as above.
+//   CTA pair, wide: output tile 256 x 512 as two 256-column halves; each CTA loads its 128 rows of
+//                opA and 128 opB rows per half, and every opA slice feeds two MMAs (one per half):
+//                a quarter fewer operand bytes per FLOP than the 256 x 256 tile. The halves are
+//                the two 256-column slots of tensor memory (one accumulator); the epilogue drains
+//                half 0 first, so the next tile's half-0 MMAs overlap the drain of half 1.
+template <bool PAIR, bool WIDE = false>
 struct TcCfg {
+  static_assert(PAIR || !WIDE, "the wide tile is a CTA-pair tile");
   static constexpr int kTileM = PAIR ? 256 : 128;
-  static constexpr int kTileN = 256;
-  static constexpr int kBRows = PAIR ? 128 : 256;
-  static constexpr int kStages = PAIR ? 6 : 4;
+  static constexpr int kTileN = WIDE ? 512 : 256;
+  static constexpr int kHalves = WIDE ? 2 : 1;
+  static constexpr int kBRows = PAIR ? 128 * kHalves : 256;
+  static constexpr int kStages = PAIR ? (WIDE ? 4 : 6) : 4;
   static constexpr uint32_t kABytes = 128 * kTcBK * 2;
+  static constexpr uint32_t kBHalfBytes = 128 * kTcBK * 2;   // 128 opB rows (CTA pair)
   static constexpr uint32_t kBBytes = kBRows * kTcBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kTmemCols = 2 * kTileN;
+  static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kEpiArrivals = PAIR ? 8 : 4;
   // CTA pair: per epilogue warp two staging sets (direct + mirrored 32 x 32 bf16 sub-tiles)
   static constexpr uint32_t kStagingPerWarp = 2 * 2 * 2048;
@@ -64,11 +73,11 @@ __device__ __forceinline__ uint32_t sw64_chunk(uint32_t r, uint32_t j) {
   return r * 64u + ((j ^ ((r >> 1) & 3u)) << 4);
 }
 
-template <bool PAIR>
+template <bool PAIR, bool WIDE>
 __global__ void __launch_bounds__(kThreads, 1)
     ns_gemm_tc_kernel(const GemmProblem* __restrict__ probs, int nprobs, uint32_t total_tiles,
                       EpiScalars ep, int* __restrict__ status) {
-  using C = TcCfg<PAIR>;
+  using C = TcCfg<PAIR, WIDE>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -131,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const GemmProblem& P = probs[tl.p];
         const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
         const int32_t a_row0 = (int32_t)(tl.bi * C::kTileM + rank * 128);
-        const int32_t b_row0 = (int32_t)(tl.bj * C::kTileN + rank * C::kBRows);
+        // single CTA: all 256 opB rows of the tile; pair: this CTA's 128 rows of each 256-wide half
+        const int32_t b_row0 = (int32_t)(tl.bj * C::kTileN + rank * (PAIR ? 128 : 0));
         for (uint32_t kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
             timed_out = true;
@@ -150,11 +160,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int h = 0; h < 2; ++h)
                 tma_load_2d_pair(a_dst + h * kBoxBytes, P.tma_a, bar, a_row0 + 64 * h, k0);
             }
-            if (!P.b_mn) {
-              tma_load_2d_pair(b_dst, P.tma_b, bar, k0, b_row0);
-            } else {
-              for (int h = 0; h < C::kBRows / 64; ++h)
-                tma_load_2d_pair(b_dst + h * kBoxBytes, P.tma_b, bar, b_row0 + 64 * h, k0);
+#pragma unroll
+            for (int hf = 0; hf < C::kHalves; ++hf) {
+              uint8_t* bh = b_dst + hf * C::kBHalfBytes;
+              const int32_t brow = b_row0 + 256 * hf;
+              if (!P.b_mn) {
+                tma_load_2d_pair(bh, P.tma_b, bar, k0, brow);
+              } else {
+                for (int h = 0; h < 2; ++h)
+                  tma_load_2d_pair(bh + h * kBoxBytes, P.tma_b, bar, brow + 64 * h, k0);
+              }
             }
           } else {
             mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
@@ -191,38 +206,94 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
         const GemmProblem& P = probs[tl.p];
         const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
-        const uint32_t idesc = idesc_bf16_f32(C::kTileM, C::kTileN, P.a_mn, P.b_mn);
+        // every MMA is kTileM x 256 x 16 (the wide tile issues one per half)
+        const uint32_t idesc = idesc_bf16_f32(C::kTileM, 256, P.a_mn, P.b_mn);
         const uint32_t a_lbo = P.a_mn ? kBoxBytes : 16u, b_lbo = P.b_mn ? kBoxBytes : 16u;
         const uint32_t a_kstep = P.a_mn ? 16u * 128u : 32u, b_kstep = P.b_mn ? 16u * 128u : 32u;
-        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
-          timed_out = true;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * C::kTileN;
-        for (uint32_t kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
-            timed_out = true;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b_addr = a_addr + C::kABytes;
+        // the MMAs of one K slice (64 deep) for one 256-column half
+        auto issue = [&](uint32_t stg, int hf, bool first_slice) {
+          const uint32_t a_addr = smem_u32(smem + stg * C::kStageBytes);
+          const uint32_t b_addr = a_addr + C::kABytes + hf * C::kBHalfBytes;
+          const uint32_t d_tmem = tmem_base + (WIDE ? hf : acc) * 256u;
 #pragma unroll
           for (uint32_t k = 0; k < kTcBK / 16; ++k) {
             const uint64_t ad = smem_desc_sw128(a_addr + k * a_kstep, a_lbo, 1024);
             const uint64_t bd = smem_desc_sw128(b_addr + k * b_kstep, b_lbo, 1024);
-            if constexpr (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, (kb | k) != 0u);
-            else tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0u);
+            const uint32_t accumulate = (!first_slice || k != 0u) ? 1u : 0u;
+            if constexpr (PAIR) tc_mma_f16_pair(d_tmem, ad, bd, idesc, accumulate);
+            else tc_mma_f16(d_tmem, ad, bd, idesc, accumulate);
           }
-          if constexpr (PAIR) tc_commit_pair_mc(&empty[stage], 0x3);
-          else tc_commit(&empty[stage]);
-          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        };
+        auto release = [&](uint32_t stg) {
+          if constexpr (PAIR) tc_commit_pair_mc(&empty[stg], 0x3);
+          else tc_commit(&empty[stg]);
+        };
+        if constexpr (!WIDE) {
+          if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+            timed_out = true;
+            break;
+          }
+          tc_fence_after();
+          for (uint32_t kb = 0; kb < kblocks; ++kb) {
+            if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
+              timed_out = true;
+              break;
+            }
+            tc_fence_after();
+            issue(stage, 0, kb == 0);
+            release(stage);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          }
+          if (timed_out) break;
+          if constexpr (PAIR) tc_commit_pair_mc(&tfull[acc], 0x3);
+          else tc_commit(&tfull[acc]);
+          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        } else {
+          // Half 0 may start as soon as the epilogue has drained half 0 of the previous tile:
+          // the first (up to kStages) resident K slices feed half 0 only; once half 1 is free
+          // too, the same slices feed half 1 and are released, then both halves go together.
+          if (!mbar_wait_bounded(&tempty[0], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+            timed_out = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t npre = kblocks < (uint32_t)C::kStages ? kblocks : (uint32_t)C::kStages;
+          uint32_t st = stage, ph = phase;
+          for (uint32_t i = 0; i < npre; ++i) {
+            if (!mbar_wait_bounded(&full[st], ph, abort_flag, kTimeoutNs)) {
+              timed_out = true;
+              break;
+            }
+            tc_fence_after();
+            issue(st, 0, i == 0);
+            if (++st == C::kStages) { st = 0; ph ^= 1u; }
+          }
+          if (timed_out) break;
+          if (!mbar_wait_bounded(&tempty[1], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+            timed_out = true;
+            break;
+          }
+          tc_fence_after();
+          for (uint32_t i = 0; i < npre; ++i) {
+            issue(stage, 1, i == 0);
+            release(stage);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          }
+          for (uint32_t kb = npre; kb < kblocks; ++kb) {
+            if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
+              timed_out = true;
+              break;
+            }
+            tc_fence_after();
+            issue(stage, 0, false);
+            issue(stage, 1, false);
+            release(stage);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          }
+          if (timed_out) break;
+          tc_commit_pair_mc(&tfull[0], 0x3);   // the whole tile (both halves)
+          acc_phase ^= 1u;
         }
-        if (timed_out) break;
-        if constexpr (PAIR) tc_commit_pair_mc(&tfull[acc], 0x3);
-        else tc_commit(&tfull[acc]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
       // all issued MMAs must finish before the tensor memory is freed
       if constexpr (PAIR) tc_commit_pair(drain);
@@ -251,8 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha = ep.e_acc ? *P.alpha : 1.0f;
       const float s1 = ep.k_acc * alpha_pow(alpha, ep.e_acc);
       const bool has_c = P.tma_c != nullptr && ep.k_c != 0.0f;
+      // the wide tile completes both halves at once, on tfull[0]
       const bool ok = __all_sync(0xffffffffu,
-                                 mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kTimeoutNs));
+                                 mbar_wait_bounded(&tfull[WIDE ? 0 : acc], acc_phase, abort_flag, kTimeoutNs));
       if (!ok) {
         timed_out = true;
         break;
@@ -263,12 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ch = 0; ch < C::kTileN / 32; ++ch) {
         uint32_t r[32];
         __syncwarp();
-        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + acc * C::kTileN + ch * 32, r);
+        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + (WIDE ? 0u : acc * 256u) + ch * 32, r);
         tmem_ld_wait();
-        if (ch == C::kTileN / 32 - 1) {
+        // a 256-column slot is free once its last chunk is in registers (wide: half 0 after
+        // chunk 7, so the next tile's half-0 MMAs can start while half 1 drains)
+        if (ch % 8 == 7) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[WIDE ? ch / 8 : acc]), 0));
         }
         const int32_t c0 = (int32_t)(tl.bj * C::kTileN + ch * 32);
         if (r0 >= (int32_t)P.M || c0 >= (int32_t)P.N) continue;        // fully clipped
@@ -371,7 +445,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         set ^= 1u;
       }
       if (timed_out) break;
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if constexpr (WIDE) {
+        acc_phase ^= 1u;
+      } else if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
@@ -486,23 +565,26 @@ cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_
   using C = TcCfg<false>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   if (total_tiles == 0) return cudaSuccess;
   if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
-  ns_gemm_tc_kernel<false><<<grid, kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status);
+  ns_gemm_tc_kernel<false, false><<<grid, kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
-                                EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
-  using C = TcCfg<true>;
+namespace {
+
+template <bool WIDE>
+cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles, EpiScalars ep,
+                        int* status, int max_pairs, cudaStream_t s) {
+  using C = TcCfg<true, WIDE>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
@@ -521,13 +603,26 @@ cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t t
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ns_gemm_tc_kernel<true>, probs, nprobs, total_tiles, ep, status);
+  return cudaLaunchKernelEx(&cfg, ns_gemm_tc_kernel<true, WIDE>, probs, nprobs, total_tiles, ep, status);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
+                                EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
+  return launch_pair<false>(probs, nprobs, total_tiles, ep, status, max_pairs, s);
+}
+
+cudaError_t launch_gemm_tc_pair_wide(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
+                                     EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
+  return launch_pair<true>(probs, nprobs, total_tiles, ep, status, max_pairs, s);
 }
 
 // Largest number of CTA pairs of the paired kernel that can be resident at once.
 int gemm_tc_pair_capacity(int sms) {
   using C = TcCfg<true>;
-  cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  static_assert(TcCfg<true, true>::kSmemBytes == C::kSmemBytes, "both pair variants have one occupancy");
+  cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::kSmemBytes);
   if (e != cudaSuccess) return sms / 2;
   cudaLaunchConfig_t cfg = {};
@@ -542,7 +637,7 @@ int gemm_tc_pair_capacity(int sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, ns_gemm_tc_kernel<true>, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&n, ns_gemm_tc_kernel<true, false>, &cfg);
   if (e != cudaSuccess || n <= 0) {
     cudaGetLastError();
     return sms / 2;

@@ -225,3 +225,40 @@ def test_step_many_matrices_multi_chunk_tables(prec, tol):
         O_gpu = (p0[j].astype(np.float64) - host64(ps[j])) / np.float64(np.float32(0.02))
         assert rel(O_gpu, O_ref) <= tol, (j, rel(O_gpu, O_ref))
         assert rel(host64(ms[j]), o_m) <= TOL_M, j
+
+
+@pytest.mark.parametrize("shape", [(2100, 3000), (3000, 2100), (2304, 2344)], ids=lambda s: f"{s[0]}x{s[1]}")
+def test_ns_wide_tiles_ragged(shape):
+    """Matrices with min(rows, cols) >= 2048 run their Gram and update products on 256 x 512 tiles:
+    ragged row and column counts (not multiples of 256 or 512), wide and tall, against the oracle."""
+    import newton_schulz_13_b200 as ns
+    G = synth.round_to(_gen(shape, 41, (1e-2, 1.0)), "bf16")
+    X = ns.ns_orthogonalize(to_dev(G, torch.bfloat16), steps=5, coeffs=Q5, eps=1e-7, prec="bf16",
+                            out_dtype=torch.float32)
+    assert ns.check_status() == ns.OK
+    want = oracle.newton_schulz(G, Q5, eps=1e-7)
+    assert rel(host64(X), want) <= TOL_O_BF16, rel(host64(X), want)
+
+
+def test_step_wide_tiles_fused_update_ragged():
+    """The fused parameter update on 256 x 512 tiles with ragged edges (2100 x 2600, tall 2600 x 2100)."""
+    import newton_schulz_13_b200 as ns
+    shapes = [(2100, 2600), (2600, 2100)]
+    rng = np.random.default_rng(43)
+    p0 = [synth.round_to(0.02 * rng.standard_normal(s), "fp32") for s in shapes]
+    g = [synth.round_to(rng.standard_normal(s), "bf16") for s in shapes]
+    ps = [to_dev(x, torch.float32) for x in p0]
+    ms = [torch.zeros(s, dtype=torch.float32, device="cuda") for s in shapes]
+    ns.muon_step(ps, [to_dev(x, torch.bfloat16) for x in g], ms, lr=0.02, mu=0.95, nesterov=True,
+                 weight_decay=0.1, rms_scale=1, steps=5, coeffs=Q5, eps=1e-7, prec="bf16")
+    torch.cuda.synchronize()
+    assert ns.check_status() == ns.OK
+    decay = np.float64(np.float32(1.0 - np.float32(0.02) * np.float32(0.1)))
+    for j, s in enumerate(shapes):
+        o_p, o_m = p0[j].astype(np.float64).copy(), np.zeros(s)
+        O_ref = oracle.muon_step([o_p], [g[j]], [o_m], lr=0.02, mu=0.95, nesterov=True, weight_decay=0.1,
+                                 rms_mode=1, coeffs=Q5, zero_center=False, eps=1e-7, want_O=True)[0]
+        rms = np.sqrt(max(1.0, s[0] / s[1]))
+        O_gpu = (p0[j] * decay - host64(ps[j])) / (np.float64(np.float32(0.02)) * rms)
+        assert rel(O_gpu, O_ref) <= TOL_O_BF16, (j, rel(O_gpu, O_ref))
+        assert rel(host64(ps[j]), o_p) <= TOL_P, j
