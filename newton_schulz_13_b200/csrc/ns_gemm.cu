@@ -86,8 +86,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;                       // followed by 4 addend-load barriers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 5);
+  uint64_t* drain = tempty + 2;                       // followed by 8 operand-load barriers
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* zero_flag = abort_flag + 1;
 
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], C::kEpiArrivals);
     }
     mbar_init(drain, 1);
-    for (int w = 0; w < 4; ++w) mbar_init(drain + 1 + w, 1);
+    for (int w = 0; w < 8; ++w) mbar_init(drain + 1 + w, 1);
     *abort_flag = 0;
     *zero_flag = 0;
     fence_mbar_init();
@@ -311,10 +311,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // also staged transposed and stored at the mirrored position, sub-tiles strictly below are
     // skipped (their mirror writes them) and diagonal sub-tiles are stored whole. Rows and
     // columns past the matrix are clipped by the TMA store.
+    // Sub-tiles alternate between two staging sets. When the epilogue reads an operand sub-tile
+    // (the addend, or the parameters of the fused update), the load of the tile's next active
+    // sub-tile goes out into the other set before this one's arithmetic, so its latency overlaps.
     const uint32_t quarter = (uint32_t)(warp & 3);
     uint8_t* stg = staging + (uint32_t)(warp - 2) * C::kStagingPerWarp;
-    uint64_t* cbar = drain + 1 + (warp - 2);    // this warp's addend-load barrier
-    uint32_t set = 0, cphase = 0;
+    uint64_t* cbar = drain + 1 + 2 * (warp - 2);   // this warp's operand-load barriers, one per set
+    uint32_t set = 0, cph = 0;                     // cph bit s: phase of cbar[s]
+    uint32_t inflight = 0;                         // bit s: a load into set s not yet waited for
+    int pend = -1;                                 // sub-tile whose load was issued ahead
     uint32_t acc = 0, acc_phase = 0;
     for (uint32_t t = unit; t < total_tiles; t += n_units) {
       const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
@@ -331,6 +336,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int32_t r0 = (int32_t)(tl.bi * C::kTileM + rank * 128 + quarter * 32);
+      // sub-tiles that produce output (the same for every lane)
+      auto active = [&](int c) {
+        const int32_t cc = (int32_t)(tl.bj * C::kTileN + c * 32);
+        return r0 < (int32_t)P.M && cc < (int32_t)P.N && !(P.sym && cc + 32 <= r0);
+      };
+      auto next_active = [&](int c) {
+        int nx = c + 1;
+        while (nx < C::kTileN / 32 && !active(nx)) ++nx;
+        return nx < C::kTileN / 32 ? nx : -1;
+      };
+      const bool loads = ep.fused != 0 || has_c;
+      const uint32_t load_bytes = ep.fused ? 4096u : 2048u;
+      const CUtensorMap* load_map = ep.fused ? P.tma_p : P.tma_c;
+      auto issue_load = [&](int c, uint32_t st) {   // lane 0
+        mbar_arrive_expect_tx(&cbar[st], load_bytes);
+        tma_load_2d(stg + st * 4096u, load_map, &cbar[st], (int32_t)(tl.bj * C::kTileN + c * 32), r0);
+      };
 #pragma unroll 1
       for (int ch = 0; ch < C::kTileN / 32; ++ch) {
         uint32_t r[32];
@@ -353,19 +375,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* mirr = direct + 2048u;
         if (lane == 0) bulk_wait_group_read<1>();   // the store issued from this set has read it
         __syncwarp();
-        if (ep.fused) {
-          // last update: the whole 4 KB set holds the 32 x 32 fp32 parameter sub-tile (128-byte
-          // swizzle); O stays in fp32 and is never stored
+        if (loads) {
+          const int nx = next_active(ch);
           if (lane == 0) {
-            mbar_arrive_expect_tx(cbar, 4096u);
-            tma_load_2d(direct, P.tma_p, cbar, c0, r0);
+            if (pend != ch) issue_load(ch, set);
+            if (nx >= 0) {
+              bulk_wait_group_read<0>();   // the other set's last store has read it too
+              issue_load(nx, set ^ 1u);
+            }
           }
-          const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(cbar, cphase, abort_flag, kTimeoutNs));
-          cphase ^= 1u;
+          inflight |= 1u << set;
+          if (nx >= 0) inflight |= 1u << (set ^ 1u);
+          pend = nx;
+          const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&cbar[set], (cph >> set) & 1u, abort_flag,
+                                                                     kTimeoutNs));
           if (!got) {
             timed_out = true;
             break;
           }
+          cph ^= 1u << set;
+          inflight &= ~(1u << set);
+        }
+        if (ep.fused) {
+          // last update: the whole 4 KB set holds the 32 x 32 fp32 parameter sub-tile (128-byte
+          // swizzle); O stays in fp32 and is never stored
           const float step = ep.lr * P.rms * s1;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -391,16 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = s1 * __uint_as_float(r[i]);
         if (has_c) {
-          if (lane == 0) {
-            mbar_arrive_expect_tx(cbar, 2048u);
-            tma_load_2d(direct, P.tma_c, cbar, c0, r0);
-          }
-          const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(cbar, cphase, abort_flag, kTimeoutNs));
-          cphase ^= 1u;
-          if (!got) {
-            timed_out = true;
-            break;
-          }
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint4 raw = *reinterpret_cast<const uint4*>(direct + sw64_chunk((uint32_t)lane, (uint32_t)j));
@@ -452,6 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    // loads still in flight (only after a timeout) must land before the CTA exits
+    if (lane == 0)
+      for (uint32_t st = 0; st < 2; ++st)
+        if (inflight & (1u << st)) mbar_wait_bounded(&cbar[st], (cph >> st) & 1u, zero_flag, kTimeoutNs);
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
   } else {
