@@ -57,13 +57,21 @@ def kernel_source_hash() -> str:
     other declarations there do not count."""
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p) as f:
+            h.update(_code_only(f.read()).encode())
     text = open(KERNEL_HEADER).read()
     for name in ("struct GemmProblem {", "struct EpiScalars {"):
         start = text.index(name)
-        h.update(text[start:text.index("};", start) + 2].encode())
+        h.update(_code_only(text[start:text.index("};", start) + 2]).encode())
     return h.hexdigest()[:16]
+
+
+def _code_only(src: str) -> str:
+    """C++ source without comments and with whitespace collapsed: edits to comments or layout do
+    not change the kernel, so they do not invalidate a recorded profile."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
 
 
 def recorded_traffic():

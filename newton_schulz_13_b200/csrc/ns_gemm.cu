@@ -2,19 +2,27 @@
 // B = b A + c A A, X = a X + B X; "AdamW vs Muon" part 3 writes the same iteration as
 // M_k = a M + b (M M^T) M + c (M M^T)^2 M).
 //
-// One kernel serves all three products. A launch is a list of independent problems (one per
-// matrix of the optimizer step, all at the same iteration and phase), each
-//     D = s_acc * (opA . opB^T) + s_c * C,
-// tiled 128 x 256 and scheduled statically over a persistent grid of one CTA per SM:
-//   warp 0      TMA producer: 64-deep K slices of opA and opB into a 4-stage smem ring
-//               (128-byte swizzle), either K-major boxes or MN-major boxes per operand;
-//   warp 1      tcgen05.mma issuer (one thread): 128 x 256 x 16 bf16 MMAs accumulating in fp32
-//               in tensor memory, two accumulators so the epilogue of one tile overlaps the
-//               MMAs of the next;
+// One kernel template serves all three products. A launch is a list of independent problems (one
+// per matrix of a wave of the optimizer step, all at the same iteration and phase), each
+//     D = s_acc * (opA . opB^T) + s_c * C + diag I,
+// scheduled statically over a persistent grid. The Muon step uses the CTA-pair variants
+// (clusters of two CTAs on two SMs, tcgen05 cta_group::2): 256 x 256 tiles, or 256 x 512 "wide"
+// tiles for the Gram and update products of large matrices. A single-CTA variant (128 x 256
+// tiles) serves the no-allocation entry point. 192 threads per CTA:
+//   warp 0      TMA producer: 64-deep K slices of opA and opB into a shared-memory ring
+//               (128-byte swizzle), K-major or MN-major boxes per operand; in a pair each CTA
+//               loads its own 128 opA rows and its 128 of every 256 opB rows, and both CTAs'
+//               copies complete on the even CTA's barrier;
+//   warp 1      tcgen05.mma issuer (one thread of the even CTA in a pair): bf16 MMAs with fp32
+//               accumulation in tensor memory; 256 x 256 tiles alternate between two
+//               accumulators, so the epilogue of one tile overlaps the MMAs of the next, and
+//               wide tiles use both 256-column slots as the two halves of one accumulator;
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, add s_c * C, round to bf16,
-//               store. For the symmetric products (A = X X^T and A A = A A^T) only tiles that
-//               touch the upper triangle are computed and the strictly-upper part is also
-//               written mirrored.
+//               stage 32 x 32 sub-tiles in shared memory and write them with TMA stores (pair),
+//               or store directly (single CTA). For the symmetric products (A = X X^T and
+//               A A = A A^T) only tiles that touch the upper triangle are computed, and the
+//               strictly-upper part is also written mirrored. The last update of a Muon step
+//               applies the parameter update instead of storing D.
 // Both orientations of the iterate are read in place: a wide iterate X (m x n) is K-major for
 // X X^T and MN-major as the right operand of B X; a tall stored matrix G (n x m, iterate G^T)
 // is MN-major for G^T G and K-major for G B. So no transposed copies are ever made.
