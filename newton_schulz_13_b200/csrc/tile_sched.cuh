@@ -1,6 +1,7 @@
-// Static tile schedule of the grouped tensor-core product kernels. A launch is a list of
-// independent problems; problem p owns the tile indices [tile_begin, tile_begin + n_tiles), and
-// the persistent grid walks the global tile index with a stride of the number of CTAs (or pairs).
+// Static tile schedule of the grouped tensor-core product kernels (and one epilogue helper they
+// share). A launch is a list of independent problems; problem p owns the tile indices
+// [tile_begin, tile_begin + n_tiles), and the persistent grid walks the tile index with a stride
+// of the number of CTAs (or pairs).
 #pragma once
 #include <stdint.h>
 
@@ -48,6 +49,7 @@ __device__ __forceinline__ Tile decode_tile(const Prob* __restrict__ probs, int 
   return tl;
 }
 
+// alpha^e for the small exponents of the epilogue scalars (e = 0, 1, 2)
 __device__ __forceinline__ float alpha_pow(float alpha, int e) {
   float s = 1.0f;
   for (int i = 0; i < e; ++i) s *= alpha;
