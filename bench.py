@@ -159,6 +159,11 @@ def reduce_max(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def all_ranks_ok(ok: bool, world: int, device=None) -> bool:
+    """True on every rank when ok is true on every rank (one collective, taken by all ranks)."""
+    return reduce_max(0.0 if ok else 1.0, world, device) == 0.0
+
+
 def barrier(world: int, device=None):
     if world == 1:
         return
@@ -399,8 +404,18 @@ def run_e2e(args, wl, step, params, grads, mom, hp, stream, world, device):
     stream as soon as its call has finished. With --sharded the whole step is one call."""
     import torch
     import newton_schulz_13_b200 as ns
-    h_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
-    h_params = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
+    # pinned host copies of the step's inputs and results (42 GB per rank for Llama-8B); every rank
+    # learns whether all of them got theirs before any collective of the measurement
+    why = None
+    try:
+        h_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
+        h_params = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
+    except RuntimeError as e:
+        h_grads = h_params = None
+        why = f"pinned host allocation failed: {str(e).splitlines()[0][:200]}"
+    if not all_ranks_ok(why is None, world, device):
+        return {"value": None, "unit": "matrices/s",
+                "unavailable": why or "pinned host allocation failed on another rank"}
     for hg, g in zip(h_grads, grads):
         hg.copy_(g)
     bi = sum(g.numel() * g.element_size() for g in grads)

@@ -46,8 +46,35 @@ def test_reduce_max_over_two_gloo_ranks():
     assert res == [(0, 15.0, 2, 0), (1, 15.0, 2, 1)]
 
 
+def _agree_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank 1 fails a local step (e.g. a pinned host allocation): every rank must see it
+        both = bench.all_ranks_ok(rank != 1, world)
+        fine = bench.all_ranks_ok(True, world)
+        q.put((rank, both, fine))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_all_ranks_ok_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_agree_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert res == [(0, False, True), (1, False, True)]
+
+
 def test_single_rank_helpers_are_identity():
     assert bench.reduce_max(3.5, 1) == 3.5
+    assert bench.all_ranks_ok(True, 1) and not bench.all_ranks_ok(False, 1)
     bench.barrier(1)
 
 
