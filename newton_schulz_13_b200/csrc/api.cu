@@ -6,11 +6,13 @@
 //   [column sums, column means]   only with zero-centring
 //   prologue                      momentum, Nesterov, norm partials, U = cast(u)
 //   norm                          alpha_j = 1 / (||u_j||_F + eps)
-//   per Newton-Schulz iteration k (one grouped launch per phase covering every matrix):
+//   per Newton-Schulz iteration k (one grouped launch per phase covering the wave's matrices):
 //     gram     A = X X^T                (k = 0: scaled by alpha^2, folding the normalisation)
 //     poly     B = b_k A + c_k A A      (skipped when c_k = 0)
 //     update   X' = a_k X + B X         (k = 0: scaled by alpha; c_k = 0: X' = a_k X + b_k A X)
-//   epilogue                      p = p (1 - lr wd) - lr s O
+//              the last update also applies p = p (1 - lr wd) - lr s O in its epilogue; a separate
+//              epilogue kernel does it only when that cannot be fused (bf16 parameters that TMA
+//              cannot view) or when steps = 0
 #include <cuda.h>
 #include <cuda_runtime.h>
 
