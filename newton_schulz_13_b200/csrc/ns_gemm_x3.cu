@@ -49,6 +49,10 @@ constexpr uint32_t kTmemCols = 2 * kTileN;
 // kept in the hi plane of D until the last one.
 constexpr uint32_t kPromote = 16;
 constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+// the 256-byte tail holds full and empty per stage, tfull and tempty per accumulator, drain, the
+// tensor-memory address and two flags
+static_assert((2 * kStages + 2 + 2 + 1) * 8 + 3 * 4 <= 256, "barrier area");
+static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA");
 
 // Shared-memory descriptor of one 8-deep K step of an operand plane: K-major tiles use the
 // 128-byte swizzle (8-row groups 1024 bytes apart); MN-major tiles the 128-byte swizzle over
