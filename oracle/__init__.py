@@ -1,8 +1,13 @@
-"""ctypes binding of the plain fp64 Muon oracle (``muon_oracle.cpp``).
+"""ctypes binding of the plain fp64 Muon oracle (``muon_oracle.cpp``), and the same method
+with library matrix products for the largest shapes (``ns_blas.py``).
 
 TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg are the only callers. The CUDA library never
 loads it, and this module never loads the CUDA library.
+
+``newton_schulz`` and ``muon_step`` take an optional ``lib``: a loaded C library (the plain-loop
+oracle, or a deliberately broken copy of it in the mutation tests), or a Python oracle module
+such as ``oracle.ns_blas`` (marked by ``PY_ORACLE = True``), which is then called directly.
 """
 from __future__ import annotations
 
@@ -63,6 +68,8 @@ def _coeff_array(coeffs: Sequence[Tuple[float, float, float]]) -> np.ndarray:
 def newton_schulz(G: np.ndarray, coeffs: Sequence[Tuple[float, float, float]], zero_center: bool = False,
                   eps: float = 1e-7, nthreads: int = 0, lib=None) -> np.ndarray:
     """O = NewtonSchulz(G) in fp64; G is rows x cols."""
+    if getattr(lib, "PY_ORACLE", False):
+        return lib.newton_schulz(G, coeffs, zero_center=zero_center, eps=eps)
     lib = lib or load()
     G = np.ascontiguousarray(G, dtype=np.float64)
     O = np.empty_like(G)
@@ -80,6 +87,10 @@ def muon_step(params: List[np.ndarray], grads: List[Optional[np.ndarray]], momen
               nthreads: int = 0, want_O: bool = False, lib=None):
     """One Muon step in fp64; params and momentum (float64, C-contiguous) are updated in place.
     Returns the list of O matrices when want_O."""
+    if getattr(lib, "PY_ORACLE", False):
+        return lib.muon_step(params, grads, momentum, lr=lr, mu=mu, nesterov=nesterov,
+                             weight_decay=weight_decay, rms_mode=rms_mode, coeffs=coeffs,
+                             zero_center=zero_center, eps=eps, want_O=want_O)
     lib = lib or load()
     n = len(params)
     for a in list(params) + list(momentum):

@@ -295,14 +295,15 @@ def pin_adamw_closed_forms(lib) -> None:
     assert np.max(np.abs(p - p0 * (1 - lr * 0.1) ** 3)) < 1e-15 and not m.any() and not v.any()
 
 
-ALL_PINS = [pin_spectral_map, pin_rank_one, pin_diagonal, pin_cubic_converges_to_polar, pin_quintic_band,
-            pin_invariances, pin_momentum_golden, pin_update_rule, pin_zero_center, pin_checkpoint_split,
-            pin_adamw_golden, pin_adamw_closed_forms]
+# the pins of the Muon step (Newton-Schulz, momentum, update); the AdamW pins follow
+MUON_PINS = [pin_spectral_map, pin_rank_one, pin_diagonal, pin_cubic_converges_to_polar, pin_quintic_band,
+             pin_invariances, pin_momentum_golden, pin_update_rule, pin_zero_center, pin_checkpoint_split]
+ALL_PINS = MUON_PINS + [pin_adamw_golden, pin_adamw_closed_forms]
 
 
-def failing_pins(lib) -> List[str]:
+def failing_pins(lib, pins: Sequence = None) -> List[str]:
     bad = []
-    for pin in ALL_PINS:
+    for pin in (ALL_PINS if pins is None else pins):
         try:
             pin(lib)
         except (AssertionError, ValueError, FloatingPointError):
