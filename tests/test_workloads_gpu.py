@@ -4,12 +4,14 @@ on its own trajectory from the same seeded inputs. No value produced by the CUDA
 to the oracle.
 
 Per step and per sampled matrix:
-  O (recovered from the device's own parameters before and after the step) <= 3e-2 (bf16 mode),
-  momentum <= 1e-6, parameters <= k * 1e-3 after k steps (the per-step bound, accumulated: the two
-  trajectories differ only through the O error of each step).
-For the Llama-8B shapes too large for the oracle (4096 x 4096, 14336 x 4096, 4096 x 14336) the
-checks are properties of the method that hold at any size:
-  - momentum element by element (the oracle with zero Newton-Schulz iterations);
+  O (recovered from the device's own parameters before and after the step) <= 3e-2 (bf16 mode)
+  or 1e-4 (fp32 mode), momentum <= 1e-6, parameters <= 1e-3 at every step (the oracle's
+  trajectory runs free: after k steps the two differ through k steps' O errors, each scaled by
+  lr ||O|| / ||p||, and the bound still holds after GPT-2-small's ten steps).
+The Llama-8B set is checked at full size on layer 0's seven matrices and on Wk, Wo and down of
+layer 31, against the fp64 oracle in its library-product form (four of those shapes take
+1.5-5.5e12 FLOP each); in bf16 mode, properties of the method that hold at any size are checked
+on top:
   - O X0^T (wide) or X0^T O (tall) is symmetric, since O = r(X0 X0^T) X0 for a polynomial r;
   - on the top singular triplets (sigma, u, v) of X0, O v = phi(sigma) u, with phi the scalar map;
   - ||O||_F^2 = sum_i phi(sigma_i)^2 over all singular values of X0.
@@ -20,6 +22,7 @@ import torch
 
 import oracle
 import synth
+from oracle import ns_blas
 from tests.gpu_util import TOL_M, TOL_O_BF16, TOL_O_FP32, TOL_P, StepCase, host64, rel, to_dev
 
 pytestmark = pytest.mark.gpu
@@ -51,7 +54,7 @@ def run_and_check(case: StepCase, n_steps: int, prec: str = "bf16", tol_o: float
             worst["O"], worst["m"], worst["p"] = max(worst["O"], e_o), max(worst["m"], e_m), max(worst["p"], e_p)
             assert e_o <= tol_o, (k, j, "O", e_o)
             assert e_m <= TOL_M, (k, j, "momentum", e_m)
-            assert e_p <= (k + 1) * TOL_P, (k, j, "params", e_p)
+            assert e_p <= TOL_P, (k, j, "params", e_p)
     import newton_schulz_13_b200 as ns
     assert ns.check_status() == ns.OK
     print(f"{wl.name} {prec}: worst O {worst['O']:.2e}, momentum {worst['m']:.2e}, params {worst['p']:.2e}")
@@ -126,87 +129,108 @@ def _top_triplets(X: np.ndarray, k: int = 6, iters: int = 80, seed: int = 0):
     return Uh[:, :k], s[:k], Vr[:, :k]
 
 
-def test_llama8b_full_size():
+# layer 0: Wq, Wk, Wv, Wo (4096 x 4096, 1024 x 4096), gate and up (14336 x 4096, the transposed
+# path, Gram contraction over 14336), down (4096 x 14336); layer 31: Wk, Wo, down
+LLAMA_SAMPLE = [0, 1, 2, 3, 4, 5, 6, 218, 220, 223]
+LLAMA_PROPS = [0, 4, 6, 220]
+# fp64 oracle results per sampled matrix (O, params, momentum as fp32 arrays: 6e-8 relative, far
+# below every tolerance) with checksums of the inputs they came from; shared by the bf16 and fp32
+# tests, which draw identical inputs
+_LLAMA_REF = {}
+
+
+def _checksum(*arrays) -> int:
+    import zlib
+    h = 0
+    for a in arrays:
+        h = zlib.crc32(np.ascontiguousarray(a).view(np.uint8), h)
+    return h
+
+
+def _llama_reference(wl, j, p_prev: np.ndarray, g: np.ndarray):
+    key = _checksum(p_prev, g)
+    if j not in _LLAMA_REF or _LLAMA_REF[j][0] != key:
+        p, m = p_prev.copy(), np.zeros_like(p_prev)
+        O = ns_blas.muon_step([p], [g], [m], lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov,
+                              weight_decay=wl.weight_decay, rms_mode=wl.rms_scale, coeffs=wl.coeffs,
+                              zero_center=False, eps=wl.eps, want_O=True)[0]
+        _LLAMA_REF[j] = (key, O.astype(np.float32), p.astype(np.float32), m.astype(np.float32))
+    return _LLAMA_REF[j][1:]
+
+
+def _llama8b_full_size(prec: str, tol_o: float, props: bool):
     import newton_schulz_13_b200 as ns
     wl = synth.WORKLOADS["llama8b"]
-    exact = [1, 2, 218]                  # Wk, Wv of layer 0; Wk of layer 31 (1024 x 4096)
-    props = [0, 4, 6, 220]               # Wq, gate (tall), down (wide) of layer 0; Wo of layer 31
-    case = StepCase(wl, sample=exact + props, device_fill=True)
-    # the oracle's full step only for the matrices it finishes in seconds
-    big = {j: case.o_params.pop(j) for j in props}
-    case.sample = exact
-    p_prev = {j: host64(case.params[j]) for j in exact + props}
-    g, O_ref = case.step(0)
+    case = StepCase(wl, sample=LLAMA_SAMPLE, device_fill=True)
+    # the reference comes from _llama_reference, not from the case's own oracle pass
+    case.sample, case.o_params, case.o_mom = [], {}, {}
+    p_prev = {j: host64(case.params[j]) for j in LLAMA_SAMPLE}
+    g, _ = case.step(0, prec=prec)
     torch.cuda.synchronize()
     assert ns.check_status() == ns.OK
     decay = np.float64(np.float32(1.0 - np.float32(wl.lr) * np.float32(wl.weight_decay)))
     lr32 = np.float64(np.float32(wl.lr))
-    for j in exact:
-        p_new = host64(case.params[j])
-        O_gpu = (p_prev[j] * decay - p_new) / (lr32 * case.rms(j))
-        assert rel(O_gpu, O_ref[j]) <= TOL_O_BF16, j
-        assert rel(p_new, case.o_params[j]) <= TOL_P, j
-        assert rel(host64(case.momentum[j]), case.o_mom[j]) <= TOL_M, j
+    worst = {"O": 0.0, "p": 0.0, "m": 0.0}
     rng = np.random.default_rng(7)
-    for j in props:
-        r, c = wl.shapes[j]
+    for j in LLAMA_SAMPLE:
         gj = host64(g[j])
-        # momentum and the normalised update X0 from the oracle with zero iterations
-        m_ref = np.zeros((r, c))
-        X0 = oracle.muon_step([big[j].copy()], [gj], [m_ref], lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov,
-                              weight_decay=wl.weight_decay, rms_mode=wl.rms_scale, coeffs=[],
-                              zero_center=False, eps=wl.eps, want_O=True)[0]
-        assert rel(host64(case.momentum[j]), m_ref) <= TOL_M, j
+        O_ref, p_ref, m_ref = _llama_reference(wl, j, p_prev[j], gj)
         p_new = host64(case.params[j])
         O = (p_prev[j] * decay - p_new) / (lr32 * case.rms(j))
-        assert np.all(np.isfinite(O))
-        tall = r > c
-        # symmetry of O X0^T (wide) or X0^T O (tall), probed with random vectors
-        R = rng.standard_normal((r if not tall else c, 16))
-        if not tall:
-            M = (O.T @ R).T @ (X0.T @ R)
-        else:
-            M = (O @ R).T @ (X0 @ R)
-        asym = np.linalg.norm(M - M.T) / np.linalg.norm(M)
-        assert asym <= 0.05, (j, "asymmetry", asym)
-        # the scalar map on the top singular triplets
-        Xo = X0 if not tall else X0.T
-        Oo = O if not tall else O.T
-        U, s, V = _top_triplets(Xo)
-        phi = scalar_map(s, wl.coeffs)
-        for i in range(len(s)):
-            resid = np.linalg.norm(Xo.T @ U[:, i] - s[i] * V[:, i]) / s[i]
-            if resid > 1e-3:
-                continue   # not converged (clustered values): skip this one
-            err = np.linalg.norm(Oo @ V[:, i] - phi[i] * U[:, i]) / phi[i]
-            assert err <= 0.05, (j, i, "triplet", err)
-        # Frobenius norm against the whole spectrum
-        sig2 = np.linalg.eigvalsh(Xo @ Xo.T)
-        want = np.sqrt(np.sum(scalar_map(np.sqrt(np.clip(sig2, 0, None)), wl.coeffs) ** 2))
-        got = np.linalg.norm(O)
-        assert abs(got / want - 1.0) <= 0.02, (j, "frobenius", got, want)
+        assert np.all(np.isfinite(O)), j
+        e_o, e_p = rel(O, O_ref), rel(p_new, p_ref)
+        e_m = rel(host64(case.momentum[j]), m_ref)
+        worst = {"O": max(worst["O"], e_o), "p": max(worst["p"], e_p), "m": max(worst["m"], e_m)}
+        assert e_o <= tol_o, (j, wl.shapes[j], "O", e_o)
+        assert e_p <= TOL_P, (j, wl.shapes[j], "params", e_p)
+        assert e_m <= TOL_M, (j, wl.shapes[j], "momentum", e_m)
+        if props and j in LLAMA_PROPS:
+            _check_properties(wl, j, gj, O, rng)
+    print(f"llama8b {prec}: worst O {worst['O']:.2e}, params {worst['p']:.2e}, momentum {worst['m']:.2e}")
+
+
+def _check_properties(wl, j, gj, O, rng):
+    r, c = wl.shapes[j]
+    # the normalised update X0 from the oracle with zero iterations
+    X0 = oracle.muon_step([np.zeros((r, c))], [gj], [np.zeros((r, c))], lr=wl.lr, mu=wl.mu, nesterov=wl.nesterov,
+                          weight_decay=wl.weight_decay, rms_mode=wl.rms_scale, coeffs=[],
+                          zero_center=False, eps=wl.eps, want_O=True)[0]
+    tall = r > c
+    # symmetry of O X0^T (wide) or X0^T O (tall), probed with random vectors
+    R = rng.standard_normal((r if not tall else c, 16))
+    if not tall:
+        M = (O.T @ R).T @ (X0.T @ R)
+    else:
+        M = (O @ R).T @ (X0 @ R)
+    asym = np.linalg.norm(M - M.T) / np.linalg.norm(M)
+    assert asym <= 0.05, (j, "asymmetry", asym)
+    # the scalar map on the top singular triplets
+    Xo = X0 if not tall else X0.T
+    Oo = O if not tall else O.T
+    U, s, V = _top_triplets(Xo)
+    phi = scalar_map(s, wl.coeffs)
+    for i in range(len(s)):
+        resid = np.linalg.norm(Xo.T @ U[:, i] - s[i] * V[:, i]) / s[i]
+        if resid > 1e-3:
+            continue   # not converged (clustered values): skip this one
+        err = np.linalg.norm(Oo @ V[:, i] - phi[i] * U[:, i]) / phi[i]
+        assert err <= 0.05, (j, i, "triplet", err)
+    # Frobenius norm against the whole spectrum
+    sig2 = np.linalg.eigvalsh(Xo @ Xo.T)
+    want = np.sqrt(np.sum(scalar_map(np.sqrt(np.clip(sig2, 0, None)), wl.coeffs) ** 2))
+    got = np.linalg.norm(O)
+    assert abs(got / want - 1.0) <= 0.02, (j, "frobenius", got, want)
+
+
+def test_llama8b_full_size():
+    """The whole Llama-8B set (224 matrices, 14 waves) in bf16 working precision."""
+    _llama8b_full_size("bf16", TOL_O_BF16, props=True)
 
 
 def test_llama8b_full_size_fp32_mode():
     """The whole Llama-8B set in fp32 working precision (3xTF32 products, 14 waves sharing one
-    9.8 GB workspace region), checked against the oracle on the matrices it finishes in seconds:
-    Wk and Wv of layer 0 (first wave) and Wk of layer 31 (last wave)."""
-    import newton_schulz_13_b200 as ns
-    wl = synth.WORKLOADS["llama8b"]
-    exact = [1, 2, 218]
-    case = StepCase(wl, sample=exact, device_fill=True)
-    p_prev = {j: host64(case.params[j]) for j in exact}
-    _, O_ref = case.step(0, prec="fp32")
-    torch.cuda.synchronize()
-    assert ns.check_status() == ns.OK
-    decay = np.float64(np.float32(1.0 - np.float32(wl.lr) * np.float32(wl.weight_decay)))
-    lr32 = np.float64(np.float32(wl.lr))
-    for j in exact:
-        p_new = host64(case.params[j])
-        O_gpu = (p_prev[j] * decay - p_new) / (lr32 * case.rms(j))
-        assert rel(O_gpu, O_ref[j]) <= TOL_O_FP32, (j, rel(O_gpu, O_ref[j]))
-        assert rel(p_new, case.o_params[j]) <= TOL_P, j
-        assert rel(host64(case.momentum[j]), case.o_mom[j]) <= TOL_M, j
+    9.8 GB workspace region)."""
+    _llama8b_full_size("fp32", TOL_O_FP32, props=False)
 
 
 # ----------------------------------------------------------------------------- waves
