@@ -36,7 +36,7 @@ METRIC = "Muon step matrices/s and NS TFLOP/s (bf16) vs B200 dense tensor peak, 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ns_gemm_tc_llama8b_traffic.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "newton_schulz_13_b200", "csrc", f)
-                  for f in ("ns_gemm.cu", "ptx.cuh", "tile_sched.cuh")]
+                  for f in ("ns_gemm.cu", "ptx.cuh", "tile_sched.cuh", "pair_pipe.cuh")]
 KERNEL_HEADER = os.path.join(ROOT, "newton_schulz_13_b200", "csrc", "muon_internal.h")
 
 
@@ -217,8 +217,14 @@ def cpu_baseline(wl: synth.Workload, nthreads: int):
     desc = (f"fp64 oracle step on matrices {sample} ({', '.join('%dx%d' % wl.shapes[j] for j in sample)}) of "
             f"layer 0 in {secs:.2f} s; whole-step time extrapolated by Newton-Schulz FLOPs "
             f"({f_sample:.3g} of {f_all:.3g}) to all {wl.count} matrices")
+    # the single 256 x 512 matrix (quintic x5, one step) on one host thread: the oracle in seconds
+    one = synth.WORKLOADS["single_256x512"]
+    one_secs = min(oracle_sample_seconds(one, [0], 1) for _ in range(3))
     return {"value": wl.count / step_secs, "unit": "matrices/s", "cores": nthreads, "kind": "oracle",
-            "sample": desc, "sample_seconds": secs, "extrapolated_step_seconds": step_secs}
+            "sample": desc, "sample_seconds": secs, "extrapolated_step_seconds": step_secs,
+            "single_256x512_one_thread": {"seconds": one_secs, "threads": 1,
+                                          "sample": "one fp64 oracle Muon step of the single 256x512 "
+                                                    "matrix on one host thread (best of 3)"}}
 
 
 # ----------------------------------------------------------------------------- ours
@@ -240,13 +246,19 @@ def run_ours(args, world, rank, local):
         owner = [rank] * wl.count
     else:
         # one weight set replicated on every rank; each rank updates its share of the matrices
-        # and the updated parameters are all-gathered (strong scaling)
+        # and the updated parameters are all-gathered, group by group, overlapping the compute
+        # (strong scaling); the parameters are views of the sharded layout's flat buffer
         from newton_schulz_13_b200 import sharded
-        owner = sharded.partition(wl.shapes, world)
+        sm = sharded.ShardedMuon(wl.shapes, device)
+        owner = sm.owner
     gdt = torch.bfloat16 if wl.grad_dtype == "bf16" else torch.float32
     params, grads, mom = [], [], []
     for j in range(wl.count):
-        params.append(wl.param_torch(j, device).to(torch.float32))
+        if args.sharded:
+            sm.params[j].copy_(wl.param_torch(j, device))
+            params.append(sm.params[j])
+        else:
+            params.append(wl.param_torch(j, device).to(torch.float32))
         grads.append(wl.grad_torch(j, 0, device).to(gdt))
         mom.append(torch.zeros(wl.shapes[j], dtype=torch.float32, device=device) if owner[j] == rank else None)
     torch.cuda.synchronize()
@@ -261,7 +273,7 @@ def run_ours(args, world, rank, local):
 
     def step():
         if args.sharded:
-            sharded.sharded_muon_step(params, grads, mom, **hp)
+            sm.step(grads, mom, **hp)
         elif len(call_groups) == 1:
             ns.muon_step(params, grads, mom, **hp)
         else:

@@ -29,13 +29,16 @@
  *   - Matrices are dense, row-major, contiguous (leading dimension = cols).
  *   - Pointers named "device" must be device memory (or managed memory) of the current device.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy default stream) and
- *     never synchronise the host, except the first call with a new set of shapes (or precision,
- *     or wave budget), which allocates the library's workspace (cudaMalloc) and uploads its
- *     tables. Per-call tables (the caller's pointers) travel to the device inside kernel launch
- *     parameters, so they never wait behind the caller's own copies on a copy engine.
+ *     never synchronise the host, except a call with a list of shapes (or precision, or wave
+ *     budget) that is not among the 16 most recently used on the device: it builds a plan (a
+ *     small table allocation with cudaMalloc, uploaded once) and, when its buffers need more
+ *     than the workspace holds, grows the workspace (cudaFree and cudaMalloc, which synchronise
+ *     the device). Per-call tables (the caller's pointers) travel to the device inside kernel
+ *     launch parameters, so they never wait behind the caller's own copies on a copy engine.
  *   - muon_step processes its matrices in waves of consecutive matrices (see
  *     muon_set_wave_elements); the workspace holds one wave's buffers, about 4 bytes per element
- *     of the largest wave in bf16 working precision and 16 in fp32.
+ *     of the largest wave seen so far in bf16 working precision and 16 in fp32. Plans of
+ *     different shape lists share it.
  *   - The workspace is owned by the library, per process, and shared by all calls: calls must be
  *     ordered (same stream, or synchronised by the caller). Concurrent calls race.
  *   - Argument errors are detected before any device work is enqueued; the call then returns a
@@ -221,6 +224,16 @@ MUON_API int muon_release_workspace(void);
  * default, 2^29; negative values are rejected with MUON_ERR_INVALID_ARG. Applies to calls made
  * after it (a cached plan built with another setting is rebuilt). */
 MUON_API int muon_set_wave_elements(int64_t elements);
+
+/* Diagnostics: the time limit, in nanoseconds, of every wait inside the Newton-Schulz product
+ * kernels launched by later muon_step and muon_ns_orthogonalize calls (operand stages,
+ * accumulators, epilogue loads). A wait that runs out makes the kernel stop early, set the
+ * timeout bit of the device status word (muon_check_status then returns MUON_ERR_TIMEOUT; that
+ * call's results are invalid) and return, leaving the device usable. ns = 0 restores the default
+ * of 2 s. A limit of a few nanoseconds makes a call give up at its first wait that is not
+ * already complete: a way to exercise that failure path. (The no-allocation call keeps the
+ * default.) Returns MUON_OK. */
+MUON_API int muon_set_wait_limit_ns(uint64_t ns);
 
 /* Kernel classes counted and timed by the library, indices into muon_profile_read's arrays. */
 enum {

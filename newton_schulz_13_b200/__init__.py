@@ -31,7 +31,7 @@ CUBIC = (1.5, -0.5, 0.0)
 
 EXPORTS = ["muon_ns_orthogonalize", "muon_step", "muon_adamw_step", "muon_last_error",
            "muon_check_status", "muon_release_workspace", "muon_profile_enable", "muon_profile_read",
-           "muon_launch_count", "muon_version", "muon_set_wave_elements"]
+           "muon_launch_count", "muon_version", "muon_set_wave_elements", "muon_set_wait_limit_ns"]
 
 
 class MuonError(RuntimeError):
@@ -78,6 +78,8 @@ def _load() -> ctypes.CDLL:
     lib.muon_release_workspace.restype = ctypes.c_int
     lib.muon_set_wave_elements.restype = ctypes.c_int
     lib.muon_set_wave_elements.argtypes = [ctypes.c_int64]
+    lib.muon_set_wait_limit_ns.restype = ctypes.c_int
+    lib.muon_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.muon_profile_enable.restype = ctypes.c_int
     lib.muon_profile_enable.argtypes = [ctypes.c_int]
     lib.muon_profile_read.restype = ctypes.c_int
@@ -228,6 +230,13 @@ def set_wave_elements(elements: int = 0) -> None:
     """Largest number of elements muon_step processes in one wave of launches (0: the default,
     2^29). Results do not depend on it; see muon_set_wave_elements in include/muon.h."""
     _check(lib.muon_set_wave_elements(int(elements)))
+
+
+def set_wait_limit_ns(ns: int = 0) -> None:
+    """Time limit of the waits inside the Newton-Schulz product kernels of later calls (0: the
+    default, 2 s). A wait that runs out makes check_status() raise with ERR_TIMEOUT; a limit of a
+    few nanoseconds exercises that path. See muon_set_wait_limit_ns in include/muon.h."""
+    _check(lib.muon_set_wait_limit_ns(int(ns)))
 
 
 def profile_enable(on: bool = True) -> None:

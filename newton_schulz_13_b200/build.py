@@ -10,7 +10,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libmuon.so")
 SOURCES = ["api.cu", "elementwise.cu", "ns_gemm.cu", "ns_gemm_x3.cu", "noalloc.cu"]
-HEADERS = ["muon_internal.h", "ptx.cuh", "tile_sched.cuh"]
+HEADERS = ["muon_internal.h", "ptx.cuh", "tile_sched.cuh", "device_once.h", "pair_pipe.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

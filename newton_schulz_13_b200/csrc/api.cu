@@ -134,6 +134,7 @@ struct BufMapsX3 {   // TMA views of one two-plane fp32 buffer: K-major and MN-m
 // cap (lower SM clock at the same board power), with per-wave launch tails costing about 3 %.
 constexpr int64_t kWaveElements = int64_t(1) << 29;
 int64_t g_wave_elements = kWaveElements;   // muon_set_wave_elements
+uint64_t g_wait_ns = 0;                     // muon_set_wait_limit_ns (0: the kernels' default)
 
 // A wave: matrices [j0, j1) of the plan. Every prefix sum in the device tables (elementwise
 // chunks, column-sum items, product tiles) restarts at zero at the wave's first matrix, so a
@@ -147,12 +148,18 @@ struct Wave {
   double ex_gram = 0, ex_poly = 0, ex_upd = 0;      // executed (tile) flops per launch
 };
 
+// A plan: the layout of one list of shapes (in one working precision and wave budget), its TMA
+// descriptors and grouped problem tables. Its tables live in a small allocation of its own; the
+// per-wave buffers (iterates, A, B, column-mean scratch, norm partials) live in the device's
+// shared buffer arena, which every plan reuses (calls are ordered on the GPU). A plan is valid
+// for the arena generation it was built against.
 struct Plan {
   std::vector<Shape> shapes;
   int x_bf16 = 1;
   int64_t wave_elements = 0;
-  char* ws = nullptr;
-  size_t ws_bytes = 0;
+  uint64_t arena_gen = 0;
+  char* tab = nullptr;       // this plan's tables (cudaMalloc)
+  size_t tab_bytes = 0;
   // device tables
   MatInfo* d_mats = nullptr;
   float* d_partials = nullptr;
@@ -178,9 +185,13 @@ struct Plan {
   std::vector<uint8_t> fused_key;
 
   ~Plan() {
-    if (ws) cudaFree(ws);
+    if (tab) cudaFree(tab);
   }
 };
+
+// Plans kept per device (most recently used first). Each holds only its tables (about 2.5 KB per
+// matrix); the buffers are shared.
+constexpr size_t kMaxPlans = 16;
 
 // Per-device table of an AdamW call: one AdamTensor per tensor, rewritten (through kernel
 // parameters) only when the pointers change.
@@ -197,7 +208,10 @@ struct AdamPlan {
 
 struct DeviceState {
   std::unique_ptr<AdamPlan> adam;
-  std::unique_ptr<Plan> plan;
+  std::vector<std::unique_ptr<Plan>> plans;   // most recently used first
+  char* arena = nullptr;                      // per-wave buffers shared by every plan
+  size_t arena_bytes = 0;
+  uint64_t arena_gen = 0;                     // bumped whenever the arena moves
   int* d_status = nullptr;  // [0] flags, [1] non-finite count
   int sms = 0;
   int cc_major = 0;
@@ -230,14 +244,18 @@ int device_state(DeviceState** out) {
   return MUON_OK;
 }
 
-// Builds the workspace, TMA descriptors and grouped problem tables for a list of shapes.
+// Finds or builds the plan (TMA descriptors, grouped problem tables, buffer layout) of a list of
+// shapes, growing the shared buffer arena when the plan needs more than it holds.
 int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Plan** out) {
-  if (ds.plan && ds.plan->shapes == shapes && ds.plan->x_bf16 == x_bf16 &&
-      ds.plan->wave_elements == g_wave_elements) {
-    *out = ds.plan.get();
-    return MUON_OK;
+  for (size_t i = 0; i < ds.plans.size(); ++i) {
+    const Plan& q = *ds.plans[i];
+    if (q.shapes == shapes && q.x_bf16 == x_bf16 && q.wave_elements == g_wave_elements &&
+        q.arena_gen == ds.arena_gen) {
+      if (i > 0) std::rotate(ds.plans.begin(), ds.plans.begin() + i, ds.plans.begin() + i + 1);
+      *out = ds.plans[0].get();
+      return MUON_OK;
+    }
   }
-  ds.plan.reset();  // frees the previous workspace (cudaFree synchronises)
   std::unique_ptr<Plan> P(new Plan());
   P->shapes = shapes;
   P->x_bf16 = x_bf16;
@@ -320,9 +338,12 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     w.cm_items = cm;
     max_chunks = std::max(max_chunks, chunks);
   }
-  off = wave_region;
+  // the arena: the wave region, then the norm partials of one wave
+  const size_t o_part = wave_region;
+  const size_t arena_need = align_up(o_part + (size_t)max_chunks * 4, AL);
+  // the plan's own tables
+  off = 0;
   const size_t o_alpha = off; off = align_up(off + (size_t)n * 4, AL);
-  const size_t o_part = off; off = align_up(off + (size_t)max_chunks * 4, AL);
   const size_t o_mats = off; off = align_up(off + (size_t)n * sizeof(MatInfo), AL);
   const int maps_per = x_bf16 ? 12 : 8;   // 4 buffers x 3 views (bf16) or x 2 views (fp32)
   const size_t o_maps = off;
@@ -334,19 +355,39 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   if (x_bf16) off = align_up(off + (size_t)n * sizeof(CUtensorMap), AL);
   const size_t o_fused = off;
   off = align_up(off + (size_t)n * prob_sz, AL);
-  P->ws_bytes = off;
+  P->tab_bytes = off;
 
-  cudaError_t e = cudaMalloc(&P->ws, P->ws_bytes);
-  if (e != cudaSuccess) {
+  auto alloc_fail = [](cudaError_t e, const char* what, size_t bytes) {
     cudaGetLastError();
-    char buf[160];
-    snprintf(buf, sizeof(buf), "workspace allocation of %.3f GB failed: %s", P->ws_bytes / 1e9,
-             cudaGetErrorString(e));
+    char buf[200];
+    snprintf(buf, sizeof(buf), "%s allocation of %.3f GB failed: %s", what, bytes / 1e9, cudaGetErrorString(e));
     return fail(MUON_ERR_WORKSPACE, buf);
+  };
+  if (arena_need > ds.arena_bytes) {
+    // every cached plan points into the arena that moves: drop them (cudaFree synchronises)
+    ds.plans.clear();
+    if (ds.arena) cudaFree(ds.arena);
+    ds.arena = nullptr;
+    ds.arena_bytes = 0;
+    ++ds.arena_gen;
+    cudaError_t e = cudaMalloc(&ds.arena, arena_need);
+    if (e != cudaSuccess) {
+      ds.arena = nullptr;
+      return alloc_fail(e, "workspace", arena_need);
+    }
+    ds.arena_bytes = arena_need;
   }
-  char* W = P->ws;
+  if (ds.plans.size() >= kMaxPlans) ds.plans.pop_back();   // least recently used
+  cudaError_t e = cudaMalloc(&P->tab, P->tab_bytes);
+  if (e != cudaSuccess) {
+    P->tab = nullptr;
+    return alloc_fail(e, "plan table", P->tab_bytes);
+  }
+  P->arena_gen = ds.arena_gen;
+  char* W = ds.arena;   // buffers
+  char* T = P->tab;     // tables
   P->d_partials = reinterpret_cast<float*>(W + o_part);
-  P->d_mats = reinterpret_cast<MatInfo*>(W + o_mats);
+  P->d_mats = reinterpret_cast<MatInfo*>(T + o_mats);
   for (int j = 0; j < n; ++j) {
     P->x0.push_back(W + o_x0[j]);
     P->x1.push_back(W + o_x1[j]);
@@ -354,7 +395,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     P->B.push_back(W + o_B[j]);
     P->colmean.push_back(reinterpret_cast<float*>(W + o_cm[j]));
     P->colpart.push_back(reinterpret_cast<float*>(W + o_cp[j]));
-    P->alpha.push_back(reinterpret_cast<float*>(W + o_alpha) + j);
+    P->alpha.push_back(reinterpret_cast<float*>(T + o_alpha) + j);
   }
 
   // ---- grouped problems
@@ -375,7 +416,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     PFN_encodeTiled_t encode = get_encode();
     if (!encode) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     std::vector<CUtensorMap> maps((size_t)n * maps_per);
-    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(W + o_maps);
+    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(T + o_maps);
     int bad = 0;
     // views: 64-wide K-major boxes of 128 rows and 64 x 64 MN-major boxes (128-byte swizzle,
     // operand loads of one CTA of a pair), and 32 x 32 boxes with the 64-byte swizzle (epilogue
@@ -482,19 +523,19 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
                       &P->d_updA[0], &P->d_updA[1]};
     for (int k = 0; k < 7; ++k) {
-      *dsts[k] = W + o_prob[k];
+      *dsts[k] = T + o_prob[k];
       MUON_CUDA(cudaMemcpy(*dsts[k], lists[k]->data(), lists[k]->size() * sizeof(GemmProblem),
                            cudaMemcpyHostToDevice));
     }
     P->h_upd[0][0] = updB[0]; P->h_upd[0][1] = updB[1];
     P->h_upd[1][0] = updA[0]; P->h_upd[1][1] = updA[1];
-    P->d_pmaps = reinterpret_cast<CUtensorMap*>(W + o_pmaps);
-    P->d_fused = W + o_fused;
+    P->d_pmaps = reinterpret_cast<CUtensorMap*>(T + o_pmaps);
+    P->d_fused = T + o_fused;
   } else {
     PFN_encodeTiled_t encode = get_encode();
     if (!encode) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     std::vector<CUtensorMap> maps((size_t)n * maps_per);
-    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(W + o_maps);
+    CUtensorMap* d_maps = reinterpret_cast<CUtensorMap*>(T + o_maps);
     int bad = 0;
     // 3-D views (columns, rows, plane) of a two-plane fp32 buffer, one plane per box: 32-wide
     // K-major boxes of 128 rows (128-byte swizzle) and 32 x 32 MN-major boxes (128-byte swizzle
@@ -596,13 +637,13 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
                       &P->d_updA[0], &P->d_updA[1]};
     for (int k = 0; k < 7; ++k) {
-      *dsts[k] = W + o_prob[k];
+      *dsts[k] = T + o_prob[k];
       MUON_CUDA(cudaMemcpy(*dsts[k], lists[k]->data(), lists[k]->size() * sizeof(GemmProblemX3),
                            cudaMemcpyHostToDevice));
     }
     P->h_upd_x3[0][0] = updB[0]; P->h_upd_x3[0][1] = updB[1];
     P->h_upd_x3[1][0] = updA[0]; P->h_upd_x3[1][1] = updA[1];
-    P->d_fused = W + o_fused;
+    P->d_fused = T + o_fused;
   }
 
   // ---- per-call table template
@@ -613,8 +654,8 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     mats[j].alpha = P->alpha[j];
   }
   P->last_uploaded = mats;   // template: pointers of the call are filled in per call
-  ds.plan = std::move(P);
-  *out = ds.plan.get();
+  ds.plans.insert(ds.plans.begin(), std::move(P));
+  *out = ds.plans[0].get();
   return MUON_OK;
 }
 
@@ -742,6 +783,7 @@ int run_ns(DeviceState& ds, Plan& P, const Wave& w, const std::vector<muon_coeff
     //   poly B = c A A + b A + a I (c = 0: gram A = b alpha^2k X X^T + a I), update X' = alpha^k B X.
     EpiScalars eg{1.0f, 0.0f, first ? 2 : 0, 0, 0.0f};
     if (P.x_bf16 && c.c == 0.0f) eg = EpiScalars{c.b, 0.0f, first ? 2 : 0, 0, c.a};
+    eg.wait_ns = g_wait_ns;
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, w.fl_gram, w.ex_gram, [&] {
         return (w.wide ? launch_gemm_tc_pair_wide : launch_gemm_tc_pair)(tc(P.d_gram[p]), n, w.tiles_gram, eg,
@@ -757,6 +799,7 @@ int run_ns(DeviceState& ds, Plan& P, const Wave& w, const std::vector<muon_coeff
     EpiScalars eu;
     if (c.c != 0.0f) {
       EpiScalars ep{c.c, c.b, 0, 0, P.x_bf16 ? c.a : 0.0f};
+      ep.wait_ns = g_wait_ns;
       if (P.x_bf16) {
         e = timed_launch(MUON_KC_GEMM, s, w.fl_poly, w.ex_poly, [&] {
           return launch_gemm_tc_pair(tc(P.d_poly), n, w.tiles_poly, ep, ds.d_status, ds.pair_capacity, s);
@@ -773,6 +816,7 @@ int run_ns(DeviceState& ds, Plan& P, const Wave& w, const std::vector<muon_coeff
       upd = P.d_updA[p];
       eu = P.x_bf16 ? EpiScalars{1.0f, 0.0f, first, 0, 0.0f} : EpiScalars{c.b, c.a, first, first, 0.0f};
     }
+    eu.wait_ns = g_wait_ns;
     if (fused_last && k + 1 == co.size()) {
       upd = const_cast<void*>(fused_last);
       eu.lr = lr;
@@ -887,8 +931,13 @@ int muon_release_workspace(void) {
   auto it = g_dev.find(dev);
   if (it == g_dev.end()) return MUON_OK;
   cudaDeviceSynchronize();
-  it->second.plan.reset();
-  it->second.adam.reset();
+  DeviceState& ds = it->second;
+  ds.plans.clear();
+  if (ds.arena) cudaFree(ds.arena);
+  ds.arena = nullptr;
+  ds.arena_bytes = 0;
+  ++ds.arena_gen;
+  ds.adam.reset();
   return MUON_OK;
 }
 
@@ -897,6 +946,13 @@ int muon_set_wave_elements(int64_t elements) {
   t_err.clear();
   if (elements < 0) return fail(MUON_ERR_INVALID_ARG, "elements must be >= 0");
   g_wave_elements = elements == 0 ? kWaveElements : elements;
+  return MUON_OK;
+}
+
+int muon_set_wait_limit_ns(uint64_t ns) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  t_err.clear();
+  g_wait_ns = ns;
   return MUON_OK;
 }
 

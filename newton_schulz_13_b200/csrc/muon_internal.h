@@ -113,12 +113,15 @@ struct GemmProblemX3 {
 // (diag is applied by the CTA-pair kernels only; the bf16 CTA-pair kernel takes alpha^e_c = 1).
 // With fused set (CTA-pair kernels, last Newton-Schulz update), O = D is not stored; instead the
 // parameters become p (1 - lr wd) - lr s O, with decay = 1 - lr wd and s = rms of the problem.
+// wait_ns limits every pipeline wait of the launch (0: the kernels' default of 2 s); a wait that
+// gives up makes the launch return early with the timeout bit set in the status word.
 struct EpiScalars {
   float k_acc, k_c;
   int e_acc, e_c;
   float diag;
   float lr, decay;
   int fused;
+  uint64_t wait_ns;
 };
 
 // Per-call tables (pointer tables of a call) travel to the device inside kernel parameters, not

@@ -151,13 +151,16 @@ extern "C" int muon_ns_orthogonalize_noalloc(const void* G, muon_dtype_t g_dtype
   if (!(eps >= 0.0f) || !std::isfinite(eps)) return na_fail(MUON_ERR_INVALID_ARG, "eps must be finite and >= 0");
   if (steps < 0 || steps > MUON_MAX_NS_STEPS)
     return na_fail(MUON_ERR_INVALID_ARG, "steps must be in [0, " + std::to_string(MUON_MAX_NS_STEPS) + "]");
+  // m and n are bounded first, so that the products below cannot overflow
   const int64_t mn = std::min(m, n);
-  const int64_t ldx = (n + 7) / 8 * 8, ldm = (mn + 7) / 8 * 8;
-  if (mn > kNaMaxMinDim || m > kNaMaxElems || m * ldx > kNaMaxElems)
+  const bool fits = m <= kNaMaxElems && n <= kNaMaxElems && mn <= kNaMaxMinDim &&
+                    m * ((n + 7) / 8 * 8) <= kNaMaxElems;
+  if (!fits)
     return na_fail(MUON_ERR_INVALID_ARG,
                    "matrix " + std::to_string(m) + "x" + std::to_string(n) +
                        " exceeds the fixed scratch of the no-allocation call (needs min(m, n) <= 1024 and "
                        "m * round_up(n, 8) <= 2097152); use muon_ns_orthogonalize");
+  const int64_t ldx = (n + 7) / 8 * 8, ldm = (mn + 7) / 8 * 8;
   muon_coeffs_t co[MUON_MAX_NS_STEPS];
   for (int k = 0; k < steps; ++k) {
     co[k] = coeffs ? coeffs[k] : muon_coeffs_t{3.4445f, -4.7750f, 2.0315f};

@@ -27,13 +27,19 @@
 // X X^T and MN-major as the right operand of B X; a tall stored matrix G (n x m, iterate G^T)
 // is MN-major for G^T G and K-major for G B. So no transposed copies are ever made.
 //
-// Every wait on an mbarrier is bounded: after kTimeoutNs the waiting role sets a shared abort
-// flag and the device status word, the producer waits for its copies in flight, the MMA thread
-// waits for its MMAs, the tensor memory is freed and the CTA returns.
+// Every wait on an mbarrier is bounded. A pipeline wait (operands, accumulators, epilogue loads)
+// gives up after the launch's limit (EpiScalars::wait_ns, 2 s by default); the role then raises
+// the abort flag of its CTA and of the partner CTA, so that every other pipeline wait returns at
+// once, and the device status word is set. Before the CTAs exit, the MMA thread waits for its
+// MMAs, the producers' copies in flight are accounted for and waited for (pair_pipe.cuh), the
+// epilogue waits for its loads and stores, and the tensor memory is freed. Those drain waits
+// keep the long limit.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "device_once.h"
 #include "muon_internal.h"
+#include "pair_pipe.cuh"
 #include "ptx.cuh"
 #include "tile_sched.cuh"
 
@@ -73,6 +79,10 @@ struct TcCfg {
   static constexpr uint32_t kStagingPerWarp = 2 * 2 * 2048;
   static constexpr uint32_t kStagingBytes = PAIR ? 4 * kStagingPerWarp : 0;
   static constexpr size_t kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 256;
+  // the 256-byte tail: full and empty per stage, tfull and tempty per accumulator, drain and 8
+  // epilogue load barriers; then the tensor-memory address, two flags and the producer's fill count
+  static_assert((2 * kStages + 2 + 2 + 9) * 8 + 4 * 4 <= 256, "barrier area");
+  static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA");
 };
 
 // Byte offset of 16-byte chunk j of row r in a 32-row x 64-byte staging box laid out with the
@@ -97,10 +107,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;                       // followed by 8 operand-load barriers
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* zero_flag = abort_flag + 1;
+  volatile int* zero_flag = abort_flag + 1;   // never set: the drain waits poll it
+  volatile uint32_t* fill_count = reinterpret_cast<volatile uint32_t*>(zero_flag + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;      // 0: the CTA that issues the MMAs
+  const uint64_t wait_ns = ep.wait_ns ? ep.wait_ns : kTimeoutNs;   // pipeline waits
   const bool leader = rank == 0;
   const uint32_t unit = PAIR ? blockIdx.x / 2 : blockIdx.x;  // pair (or CTA) index
   const uint32_t n_units = PAIR ? gridDim.x / 2 : gridDim.x;
@@ -118,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int w = 0; w < 8; ++w) mbar_init(drain + 1 + w, 1);
     *abort_flag = 0;
     *zero_flag = 0;
+    *fill_count = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -142,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int issued_parity[C::kStages];
       for (int s = 0; s < C::kStages; ++s) issued_parity[s] = -1;
-      uint32_t stage = 0, phase = 0;
+      uint32_t stage = 0, phase = 0, fills = 0;
       for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
         const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
         const GemmProblem& P = probs[tl.p];
@@ -151,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // single CTA: all 256 opB rows of the tile; pair: this CTA's 128 rows of each 256-wide half
         const int32_t b_row0 = (int32_t)(tl.bj * C::kTileN + rank * (PAIR ? 128 : 0));
         for (uint32_t kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, wait_ns)) {
             timed_out = true;
             break;
           }
@@ -195,15 +208,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           issued_parity[stage] = (int)phase;
+          ++fills;
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      // copies in flight must land before this CTA's shared memory is released (the even CTA's
-      // barriers also count the odd CTA's copies)
-      if (leader)
+      if (timed_out) raise_abort(abort_flag, PAIR, rank);
+      if constexpr (PAIR) {
+        *fill_count = fills;   // settled with the partner's count at exit (pair_pipe.cuh)
+      } else {
+        // copies in flight must land before this CTA's shared memory is released
         for (int s = 0; s < C::kStages; ++s)
           if (issued_parity[s] >= 0)
             mbar_wait_bounded(&full[s], (uint32_t)issued_parity[s], zero_flag, kTimeoutNs);
+      }
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -237,13 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           else tc_commit(&empty[stg]);
         };
         if constexpr (!WIDE) {
-          if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, wait_ns)) {
             timed_out = true;
             break;
           }
           tc_fence_after();
           for (uint32_t kb = 0; kb < kblocks; ++kb) {
-            if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
+            if (!mbar_wait_bounded(&full[stage], phase, abort_flag, wait_ns)) {
               timed_out = true;
               break;
             }
@@ -260,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // Half 0 may start as soon as the epilogue has drained half 0 of the previous tile:
           // the first (up to kStages) resident K slices feed half 0 only; once half 1 is free
           // too, the same slices feed half 1 and are released, then both halves go together.
-          if (!mbar_wait_bounded(&tempty[0], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&tempty[0], acc_phase ^ 1u, abort_flag, wait_ns)) {
             timed_out = true;
             break;
           }
@@ -268,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t npre = kblocks < (uint32_t)C::kStages ? kblocks : (uint32_t)C::kStages;
           uint32_t st = stage, ph = phase;
           for (uint32_t i = 0; i < npre; ++i) {
-            if (!mbar_wait_bounded(&full[st], ph, abort_flag, kTimeoutNs)) {
+            if (!mbar_wait_bounded(&full[st], ph, abort_flag, wait_ns)) {
               timed_out = true;
               break;
             }
@@ -277,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++st == C::kStages) { st = 0; ph ^= 1u; }
           }
           if (timed_out) break;
-          if (!mbar_wait_bounded(&tempty[1], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&tempty[1], acc_phase ^ 1u, abort_flag, wait_ns)) {
             timed_out = true;
             break;
           }
@@ -288,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
           for (uint32_t kb = npre; kb < kblocks; ++kb) {
-            if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
+            if (!mbar_wait_bounded(&full[stage], phase, abort_flag, wait_ns)) {
               timed_out = true;
               break;
             }
@@ -303,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc_phase ^= 1u;
         }
       }
+      if (timed_out) raise_abort(abort_flag, PAIR, rank);
       // all issued MMAs must finish before the tensor memory is freed
       if constexpr (PAIR) tc_commit_pair(drain);
       else tc_commit(drain);
@@ -337,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool has_c = P.tma_c != nullptr && ep.k_c != 0.0f;
       // the wide tile completes both halves at once, on tfull[0]
       const bool ok = __all_sync(0xffffffffu,
-                                 mbar_wait_bounded(&tfull[WIDE ? 0 : acc], acc_phase, abort_flag, kTimeoutNs));
+                                 mbar_wait_bounded(&tfull[WIDE ? 0 : acc], acc_phase, abort_flag, wait_ns));
       if (!ok) {
         timed_out = true;
         break;
@@ -361,12 +379,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&cbar[st], load_bytes);
         tma_load_2d(stg + st * 4096u, load_map, &cbar[st], (int32_t)(tl.bj * C::kTileN + c * 32), r0);
       };
-#pragma unroll 1
-      for (int ch = 0; ch < C::kTileN / 32; ++ch) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + (WIDE ? 0u : acc * 256u) + ch * 32, r);
-        tmem_ld_wait();
+      // TMEM loads run one 32-column chunk ahead of the arithmetic: the load of the next active
+      // chunk is issued before the current chunk is processed, and waited for after it. Chunks
+      // that produce no output (clipped, or below the diagonal of a symmetric output) are not
+      // loaded at all.
+      const uint32_t tmem_row = (quarter * 32u) << 16;
+      auto tmem_col = [&](int c) { return (WIDE ? 0u : acc * 256u) + (uint32_t)c * 32u; };
+      // one chunk whose accumulator values are in r; false when an operand-load wait gave up
+      auto chunk = [&](const uint32_t (&r)[32], int ch) -> bool {
         // a 256-column slot is free once its last chunk is in registers (wide: half 0 after
         // chunk 7, so the next tile's half-0 MMAs can start while half 1 drains)
         if (ch % 8 == 7) {
@@ -375,8 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[WIDE ? ch / 8 : acc]), 0));
         }
         const int32_t c0 = (int32_t)(tl.bj * C::kTileN + ch * 32);
-        if (r0 >= (int32_t)P.M || c0 >= (int32_t)P.N) continue;        // fully clipped
-        if (P.sym && c0 + 32 <= r0) continue;                            // mirrored elsewhere
+        if (r0 >= (int32_t)P.M || c0 >= (int32_t)P.N) return true;        // fully clipped
+        if (P.sym && c0 + 32 <= r0) return true;                            // mirrored elsewhere
         const bool diag_blk = P.sym && c0 == r0;
         const bool mirror = P.sym && c0 >= r0 + 32;
         uint8_t* direct = stg + set * 4096u;
@@ -396,11 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (nx >= 0) inflight |= 1u << (set ^ 1u);
           pend = nx;
           const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&cbar[set], (cph >> set) & 1u, abort_flag,
-                                                                     kTimeoutNs));
-          if (!got) {
-            timed_out = true;
-            break;
-          }
+                                                                     wait_ns));
+          if (!got) return false;
           cph ^= 1u << set;
           inflight &= ~(1u << set);
         }
@@ -426,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit_group();
           }
           set ^= 1u;
-          continue;
+          return true;
         }
         float v[32];
 #pragma unroll
@@ -474,7 +491,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_commit_group();
         }
         set ^= 1u;
+        return true;
+      };
+      auto step = [&](const uint32_t (&cur)[32], uint32_t (&nxt)[32], int ch) -> bool {
+        __syncwarp();
+        if (ch + 1 < C::kTileN / 32 && active(ch + 1)) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(ch + 1), nxt);
+        const bool ok = chunk(cur, ch);
+        tmem_ld_wait();
+        return ok;
+      };
+      uint32_t ra[32], rb[32];
+      __syncwarp();
+      if (active(0)) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(0), ra);
+      tmem_ld_wait();
+      bool chunks_ok = true;
+#pragma unroll 1
+      for (int ch = 0; ch < C::kTileN / 32 && chunks_ok; ch += 2) {   // kTileN / 32 is even
+        chunks_ok = step(ra, rb, ch);
+        if (chunks_ok) chunks_ok = step(rb, ra, ch + 1);
       }
+      if (!chunks_ok) timed_out = true;
       if (timed_out) break;
       if constexpr (WIDE) {
         acc_phase ^= 1u;
@@ -483,6 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc_phase ^= 1u;
       }
     }
+    if (timed_out && lane == 0) raise_abort(abort_flag, PAIR, rank);
     // loads still in flight (only after a timeout) must land before the CTA exits
     if (lane == 0)
       for (uint32_t st = 0; st < 2; ++st)
@@ -503,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every lane polls; the outcome is made warp-uniform so that the warp stays converged
       // for the .sync.aligned tensor-memory loads below
       const bool ok = __all_sync(0xffffffffu,
-                                 mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kTimeoutNs));
+                                 mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, wait_ns));
       if (!ok) {
         timed_out = true;
         break;
@@ -575,17 +612,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (timed_out && lane == 0) raise_abort(abort_flag, false, rank);
   }
 
-  if (timed_out) {
-    *abort_flag = 1;
-    atomicOr(status, kStatusTimeout);
-  }
+  if (timed_out) atomicOr(status, kStatusTimeout);
   tc_fence_before();
   __syncthreads();
-  // the pair leaves together: no CTA exits while its partner may still signal its barriers or
-  // (even CTA) write its tensor memory
-  if constexpr (PAIR) cluster_sync();
+  if constexpr (PAIR) {
+    // every role of both CTAs has left its loop and the producers' fill counts are visible; the
+    // even CTA's producer accounts for the copies still in flight (pair_pipe.cuh)
+    cluster_sync();
+    if (warp == 0 && lane == 0 && leader) {
+      const uint32_t peer = ld_shared_cluster(mapa_shared(smem_u32((const void*)fill_count), 1u));
+      settle_pair_fills<C::kStages>(full, *fill_count, peer, C::kStageBytes, zero_flag, kTimeoutNs);
+    }
+    __syncwarp();
+    // the pair leaves together: no CTA exits while a copy may still land in its shared memory,
+    // or while its partner may still signal its barriers or (even CTA) write its tensor memory
+    cluster_sync();
+  }
   tc_fence_after();
   if (warp == 1) {
     if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
@@ -593,18 +638,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Raises a kernel's dynamic shared-memory limit on the current device, once per device (the
+// attribute belongs to one device's context). `once` is the kernel's own set of flags.
+cudaError_t set_smem_limit(const void* kernel, int bytes, PerDeviceOnce& once) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  return (cudaError_t)once.run(dev, [&] {
+    return (int)cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+}
+
 }  // namespace
 
 cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                            EpiScalars ep, int* status, int grid, cudaStream_t s) {
   using C = TcCfg<false>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce once;
+  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<false, false>, (int)C::kSmemBytes, once);
+  if (e != cudaSuccess) return e;
   if (total_tiles == 0) return cudaSuccess;
   if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
   ns_gemm_tc_kernel<false, false><<<grid, kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status);
@@ -617,13 +669,9 @@ template <bool WIDE>
 cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles, EpiScalars ep,
                         int* status, int max_pairs, cudaStream_t s) {
   using C = TcCfg<true, WIDE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce once;   // one per tile width
+  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<true, WIDE>, (int)C::kSmemBytes, once);
+  if (e != cudaSuccess) return e;
   if (total_tiles == 0) return cudaSuccess;
   const uint32_t pairs = (uint32_t)max_pairs < total_tiles ? (uint32_t)max_pairs : total_tiles;
   cudaLaunchConfig_t cfg = {};

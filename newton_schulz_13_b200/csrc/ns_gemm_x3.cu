@@ -22,11 +22,15 @@
 //              planes (symmetric products: the upper triangle, and the strictly-upper part again
 //              at the mirrored position); for the last update of a Muon step,
 //              p <- p decay - lr s D instead, and D is never stored.
-// Every mbarrier wait is bounded as in the bf16 kernel: on timeout the status word is set, copies
-// and MMAs in flight are drained, the tensor memory is freed and the CTAs return.
+// Every mbarrier wait is bounded as in the bf16 kernel: a pipeline wait gives up after the
+// launch's limit (EpiScalars::wait_ns, 2 s by default) and raises the abort flag of both CTAs of
+// the pair; the status word is set, copies and MMAs in flight are accounted for and drained
+// (pair_pipe.cuh), the tensor memory is freed and the CTAs return.
 #include <stdint.h>
 
+#include "device_once.h"
 #include "muon_internal.h"
+#include "pair_pipe.cuh"
 #include "ptx.cuh"
 #include "tile_sched.cuh"
 
@@ -50,8 +54,8 @@ constexpr uint32_t kTmemCols = 2 * kTileN;
 constexpr uint32_t kPromote = 16;
 constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
 // the 256-byte tail holds full and empty per stage, tfull and tempty per accumulator, drain, the
-// tensor-memory address and two flags
-static_assert((2 * kStages + 2 + 2 + 1) * 8 + 3 * 4 <= 256, "barrier area");
+// tensor-memory address, two flags and the producer's fill count
+static_assert((2 * kStages + 2 + 2 + 1) * 8 + 4 * 4 <= 256, "barrier area");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA");
 
 // Shared-memory descriptor of one 8-deep K step of an operand plane: K-major tiles use the
@@ -104,10 +108,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* zero_flag = abort_flag + 1;
+  volatile int* zero_flag = abort_flag + 1;   // never set: the drain waits poll it
+  volatile uint32_t* fill_count = reinterpret_cast<volatile uint32_t*>(zero_flag + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();   // 0: the CTA that issues the MMAs
+  const uint64_t wait_ns = ep.wait_ns ? ep.wait_ns : kTimeoutNs;   // pipeline waits
   const bool leader = rank == 0;
   const uint32_t unit = blockIdx.x / 2;
   const uint32_t n_units = gridDim.x / 2;
@@ -124,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     *zero_flag = 0;
+    *fill_count = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -141,9 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
-      int issued_parity[kStages];
-      for (int s = 0; s < kStages; ++s) issued_parity[s] = -1;
-      uint32_t stage = 0, phase = 0;
+      uint32_t stage = 0, phase = 0, fills = 0;
       for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
         const Tile tl = decode_tile<kTileM, kTileN>(probs, nprobs, t);
         const GemmProblemX3& P = probs[tl.p];
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t a_row0 = (int32_t)(tl.bi * kTileM + rank * 128);
         const int32_t b_row0 = (int32_t)(tl.bj * kTileN + rank * 128);
         for (uint32_t kb = 0; kb < kblocks; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, wait_ns)) {
             timed_out = true;
             break;
           }
@@ -165,14 +170,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             load_operand(dst + pl * kPlaneTile, P.tma_a, P.a_mn != 0, bar, a_row0, k0, pl);
             load_operand(dst + (2 + pl) * kPlaneTile, P.tma_b, P.b_mn != 0, bar, b_row0, k0, pl);
           }
-          issued_parity[stage] = (int)phase;
+          ++fills;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
         }
       }
-      if (leader)
-        for (int s = 0; s < kStages; ++s)
-          if (issued_parity[s] >= 0)
-            mbar_wait_bounded(&full[s], (uint32_t)issued_parity[s], zero_flag, kTimeoutNs);
+      if (timed_out) raise_abort(abort_flag, true, rank);
+      *fill_count = fills;   // settled with the partner's count at exit (pair_pipe.cuh)
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -190,14 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (uint32_t kb = 0; kb < kblocks; ++kb) {
           const uint32_t kc = kb % kPromote;   // position inside the current accumulation chunk
           if (kc == 0) {
-            if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, kTimeoutNs)) {
+            if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, wait_ns)) {
               timed_out = true;
               break;
             }
             tc_fence_after();
             d_tmem = tmem_base + acc * kTileN;
           }
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, kTimeoutNs)) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, wait_ns)) {
             timed_out = true;
             break;
           }
@@ -223,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (timed_out) break;
       }
+      if (timed_out) raise_abort(abort_flag, true, rank);
       tc_commit_pair(drain);
       mbar_wait_bounded(drain, 0, zero_flag, kTimeoutNs);
     }
@@ -253,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t c = 0; c < nchunks && !timed_out; ++c) {
         const bool last = c + 1 == nchunks;
         const bool ok = __all_sync(0xffffffffu,
-                                   mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, kTimeoutNs));
+                                   mbar_wait_bounded(&tfull[acc], acc_phase, abort_flag, wait_ns));
         if (!ok) {
           timed_out = true;
           break;
@@ -381,15 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (timed_out) break;
     }
+    if (timed_out && lane == 0) raise_abort(abort_flag, true, rank);
   }
 
-  if (timed_out) {
-    *abort_flag = 1;
-    atomicOr(status, kStatusTimeout);
-  }
+  if (timed_out) atomicOr(status, kStatusTimeout);
   tc_fence_before();
   __syncthreads();
-  cluster_sync();   // the pair leaves together
+  // every role of both CTAs has left its loop and the producers' fill counts are visible; the even
+  // CTA's producer accounts for the copies still in flight (pair_pipe.cuh)
+  cluster_sync();
+  if (warp == 0 && lane == 0 && leader) {
+    const uint32_t peer = ld_shared_cluster(mapa_shared(smem_u32((const void*)fill_count), 1u));
+    settle_pair_fills<kStages>(full, *fill_count, peer, kStageBytes, zero_flag, kTimeoutNs);
+  }
+  __syncwarp();
+  // the pair leaves together: no CTA exits while a copy may still land in its shared memory, or
+  // while its partner may still signal its barriers or (even CTA) write its tensor memory
+  cluster_sync();
   tc_fence_after();
   if (warp == 1) tmem_dealloc_pair(tmem_base, kTmemCols);
 }
@@ -409,13 +421,17 @@ cudaLaunchConfig_t pair_config(uint32_t pairs, cudaStream_t s, cudaLaunchAttribu
   return cfg;
 }
 
+// Raises the kernel's dynamic shared-memory limit on the current device, once per device (the
+// attribute belongs to one device's context).
 cudaError_t set_smem_attr() {
-  static bool done = false;
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(ns_gemm_x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
-  if (e == cudaSuccess) done = true;
-  return e;
+  static PerDeviceOnce once;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  return (cudaError_t)once.run(dev, [] {
+    return (int)cudaFuncSetAttribute(ns_gemm_x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kSmemBytes);
+  });
 }
 
 }  // namespace

@@ -108,6 +108,44 @@ def test_noalloc_rejects_oversize_before_device_work():
     assert f(0x1000, 1, 0x100000000, 1, 1025, 1025, 5, None, 1e-7, None, None) == ns.ERR_INVALID_ARG
     assert "scratch" in ns.last_error()
     assert f(0x1000, 1, 0x100000000, 1, 8, 1 << 20, 5, None, 1e-7, None, None) == ns.ERR_INVALID_ARG
+    # sizes whose products would overflow 64 bits are bounded before any product is formed
+    for m, n in ((8, 1 << 62), (1 << 62, 8), (8, (1 << 63) - 1), ((1 << 63) - 1, (1 << 63) - 1)):
+        assert f(0x1000, 1, 0x100000000, 1, m, n, 5, None, 1e-7, None, None) == ns.ERR_INVALID_ARG, (m, n)
+        assert "scratch" in ns.last_error()
+
+
+PER_DEVICE_ONCE_CHECK = r"""
+#include <cstdio>
+#include "device_once.h"
+int main() {
+  muon::PerDeviceOnce once;
+  int calls = 0, fail_next = 0;
+  auto fn = [&] { ++calls; if (fail_next) { fail_next = 0; return 7; } return 0; };
+  if (once.run(0, fn) != 0 || calls != 1 || !once.done(0)) return 1;
+  if (once.run(0, fn) != 0 || calls != 1) return 2;            // device 0: done, skipped
+  if (once.done(1) || once.run(1, fn) != 0 || calls != 2) return 3;   // a second device runs it
+  fail_next = 1;
+  if (once.run(70, fn) != 7 || calls != 3 || once.done(70)) return 4;  // a failure is not kept
+  if (once.run(70, fn) != 0 || calls != 4 || !once.done(70)) return 5; // and is retried
+  if (once.run(-1, fn) != 0 || once.run(-1, fn) != 0 || calls != 6) return 6;   // untracked: always
+  if (once.run(muon::PerDeviceOnce::kTracked, fn) != 0 || calls != 7) return 7;
+  if (!once.done(0) || !once.done(1) || once.done(2)) return 8;
+  std::puts("ok");
+  return 0;
+}
+"""
+
+
+def test_kernel_attributes_are_set_once_per_device(tmp_path):
+    """The bookkeeping behind the kernels' shared-memory limit (an attribute of one device's
+    context): set once per device, again on every other device, retried after a failure."""
+    src = tmp_path / "once.cpp"
+    src.write_text(PER_DEVICE_ONCE_CHECK)
+    exe = tmp_path / "once"
+    subprocess.check_call(["g++", "-std=c++17", "-Wall", "-Werror", "-I",
+                           os.path.join(ROOT, "newton_schulz_13_b200", "csrc"), str(src), "-o", str(exe)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.returncode
 
 
 @pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="checks the no-device path")

@@ -1,6 +1,8 @@
-"""Matrix-sharded Muon step: the ownership split, and the exchange that makes every replica
-agree, run on two gloo ranks on CPU with a host-side stand-in for the local CUDA step. The GPU
-test checks that one rank reproduces muon_step exactly."""
+"""Matrix-sharded Muon step: the ownership split, the grouped flat layout, and the per-group
+exchange that makes every replica agree (each group's gather issued after that group's compute
+and before the next group's), run on two gloo ranks on CPU with a host-side stand-in for the
+local CUDA step. The GPU test checks that one rank, in several groups, reproduces muon_step
+exactly."""
 import os
 import socket
 
@@ -33,31 +35,72 @@ def _free_port():
     return p
 
 
+def test_layout_places_every_matrix_in_its_group_and_owner_slot():
+    shapes = synth.WORKLOADS["llama8b"].shapes
+    for world in (1, 2, 8):
+        L = sharded.ShardedLayout(shapes, world)
+        spans = []
+        for j, (r, c) in enumerate(shapes):
+            g, o = L.group_of[j], L.offset[j]
+            slot0 = L.block_off[g] + L.owner[j] * L.cap[g]
+            assert slot0 <= o and o + r * c <= slot0 + L.cap[g], (world, j)
+            assert j in L.groups[L.owner[j]][g]
+            spans.append((o, o + r * c))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))   # no two views overlap
+        assert L.padding() < 0.08, (world, L.padding())
+        # every rank's groups are balanced to within one matrix of the group's share
+        assert L.n_groups == max(1, -(-max(sum(r * c for j, (r, c) in enumerate(shapes) if L.owner[j] == k)
+                                          for k in range(world)) // (1 << 28)))
+    with pytest.raises(ValueError):
+        sharded.ShardedLayout(shapes, 2, group_elements=0)
+
+
+def test_expected_exchange_time():
+    shapes = synth.WORKLOADS["llama8b"].shapes
+    # 28 GB of fp32 parameters; at 8 ranks each receives 7/8 of them
+    ms = sharded.expected_exchange_ms(shapes, 8, link_gbs=725.0)
+    assert 30.0 < ms < 40.0, ms
+    assert sharded.expected_exchange_ms(shapes, 1) == 0.0
+
+
 def _fake_local_step(ps, gs, ms, lr=0.1, **kw):
     for p, g, m in zip(ps, gs, ms):
         m.add_(g)
         p.sub_(lr * m)
 
 
+SHAPES = [(3, 5), (8, 8), (2, 9), (6, 4), (7, 7), (16, 3), (5, 5), (9, 2)]
+
+
 def _worker(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        shapes = [(3, 5), (8, 8), (2, 9), (6, 4), (7, 7)]
         gen = torch.Generator().manual_seed(0)
-        params = [torch.randn(s, generator=gen) for s in shapes]
-        grads = [torch.randn(s, generator=gen) for s in shapes]
-        want = [p - 0.1 * g for p, g in zip(params, grads)]
-        mom = [torch.zeros(s) for s in shapes]
-        owner = sharded.sharded_muon_step(params, grads, mom, local_step=_fake_local_step, lr=0.1)
-        ok_params = all(torch.allclose(p, w, rtol=0, atol=1e-6) for p, w in zip(params, want))
-        ok_mom = all(torch.equal(m, grads[j]) if owner[j] == rank else torch.equal(m, torch.zeros_like(m))
-                     for j, m in enumerate(mom))
-        flat = torch.cat([p.reshape(-1) for p in params])
+        init = [torch.randn(s, generator=gen) for s in SHAPES]
+        grads = [torch.randn(s, generator=gen) for s in SHAPES]
+        events = []
+        # small groups: three or more per rank, so the per-group ordering is exercised
+        sm = sharded.ShardedMuon(SHAPES, group_elements=40, local_step=_fake_local_step, on_event=events.append)
+        for p, v in zip(sm.params, init):
+            p.copy_(v)
+        mom = [torch.zeros(s) if sm.owner[j] == rank else None for j, s in enumerate(SHAPES)]
+        results = {}
+        for step in range(2):
+            sm.step(grads, mom, lr=0.1)
+            want = [v - 0.1 * (step + 1) * (step + 2) / 2 * g for v, g in zip(init, grads)]
+            results[step] = all(torch.allclose(p, w, rtol=0, atol=1e-5) for p, w in zip(sm.params, want))
+        ok_mom = all(torch.allclose(m, 2 * grads[j]) for j, m in enumerate(mom) if m is not None)
+        flat = torch.cat([p.reshape(-1) for p in sm.params])
         gathered = [torch.empty_like(flat) for _ in range(world)]
         dist.all_gather(gathered, flat)
         same = all(torch.equal(gathered[0], g) for g in gathered)
-        q.put((rank, ok_params, ok_mom, same, sorted(set(owner))))
+        G = sm.layout.n_groups
+        # per step: compute g, then its gather, then compute g + 1 ...
+        order = [("compute", g) if i % 2 == 0 else ("gather", g) for g in range(G) for i in range(2)]
+        ok_order = events == order * 2
+        q.put((rank, results[0] and results[1], ok_mom, same, ok_order, G, sorted(set(sm.owner))))
     finally:
         dist.destroy_process_group()
 
@@ -73,8 +116,10 @@ def test_exchange_on_two_gloo_ranks():
         p.join(120)
         assert p.exitcode == 0
     res = sorted(q.get(timeout=10) for _ in range(2))
-    for rank, ok_params, ok_mom, same, owners in res:
-        assert ok_params and ok_mom and same and owners == [0, 1], (rank, ok_params, ok_mom, same, owners)
+    for rank, ok_params, ok_mom, same, ok_order, G, owners in res:
+        assert G >= 3, G
+        assert ok_params and ok_mom and same and ok_order and owners == [0, 1], (rank, ok_params, ok_mom, same,
+                                                                                 ok_order, owners)
 
 
 @pytest.mark.gpu
@@ -85,11 +130,14 @@ def test_single_rank_matches_muon_step():
     gen = torch.Generator(device="cuda").manual_seed(5)
     p_a = [torch.randn(s, device="cuda", generator=gen) * 0.02 for s in shapes]
     g = [torch.randn(s, device="cuda", generator=gen).bfloat16() for s in shapes]
-    p_b = [p.clone() for p in p_a]
+    sm = sharded.ShardedMuon(shapes, "cuda", group_elements=1 << 20)
+    for p, v in zip(sm.params, p_a):
+        p.copy_(v)
     m_a = [torch.zeros(s, device="cuda") for s in shapes]
     m_b = [torch.zeros(s, device="cuda") for s in shapes]
     ns.muon_step(p_a, g, m_a, lr=0.02, weight_decay=0.01)
-    sharded.sharded_muon_step(p_b, g, m_b, lr=0.02, weight_decay=0.01)
+    sm.step(g, m_b, lr=0.02, weight_decay=0.01)
     torch.cuda.synchronize()
-    assert all(torch.equal(a, b) for a, b in zip(p_a, p_b))
+    assert sm.layout.n_groups >= 2
+    assert all(torch.equal(a, b) for a, b in zip(p_a, sm.params))
     assert all(torch.equal(a, b) for a, b in zip(m_a, m_b))

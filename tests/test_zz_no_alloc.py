@@ -4,14 +4,17 @@ It exists for callers that cannot allocate device memory while they run (a plugi
 hook whose framework owns every allocation, or a service that reserves its memory at start-up):
 it works in a fixed scratch array compiled into the library instead of a cudaMalloc'd
 workspace. These tests call it through the C ABI and compare it with the allocating
-muon_ns_orthogonalize on two calls in a row, within the bf16 tolerance the other parity tests
-use. This file is named to be collected last.
+muon_ns_orthogonalize on two calls in a row, and with the fp64 oracle, within the bf16
+tolerance the other parity tests use, including matrices at the limits of the scratch layout.
+This file is named to be collected last.
 """
 import ctypes
 
 import numpy as np
 import pytest
 import torch
+
+from oracle import ns_blas
 
 pytestmark = pytest.mark.gpu
 
@@ -63,6 +66,8 @@ def test_noalloc_matches_allocating_entry_point_on_two_calls():
         assert status.tolist() == [0, 0]
         assert torch.isfinite(X_na).all()
         assert _rel(X_na, X_ref) <= TOL_O_BF16
+        want = ns_blas.newton_schulz(G.double().cpu().numpy(), co, eps=1e-7)
+        assert _rel(X_na.cpu(), torch.from_numpy(want)) <= TOL_O_BF16
 
 
 def test_noalloc_call_does_not_grow_device_memory_and_rejects_oversize():
@@ -84,3 +89,44 @@ def test_noalloc_call_does_not_grow_device_memory_and_rejects_oversize():
     out = torch.empty_like(big)
     rc = f(big.data_ptr(), ns.FP32, out.data_ptr(), ns.FP32, 1100, 1100, 5, co, 1e-7, None, stream)
     assert rc == ns.ERR_INVALID_ARG and "scratch" in ns.last_error()
+
+
+# the largest accepted sizes in both orientations (min(m, n) = 1024, m * round_up(n, 8) = 2^21),
+# a ragged one just under the limit (1016 * 2056 = 2,088,896 elements), a bf16 output and steps = 0
+LIMIT_CASES = [((1024, 2048), torch.float32, torch.float32, 5),
+               ((2048, 1024), torch.bfloat16, torch.bfloat16, 5),
+               ((1016, 2050), torch.float32, torch.bfloat16, 5),
+               ((2050, 1016), torch.bfloat16, torch.float32, 5),
+               ((300, 700), torch.float32, torch.float32, 0)]
+
+
+@pytest.mark.parametrize("shape,gdt,xdt,steps", LIMIT_CASES,
+                         ids=lambda v: "x".join(map(str, v)) if isinstance(v, tuple) else str(v))
+def test_noalloc_at_the_scratch_limits(shape, gdt, xdt, steps):
+    ns, f = _entry()
+    stream = torch.cuda.current_stream().cuda_stream
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    r, c = shape
+    gen = torch.Generator(device="cuda").manual_seed(r * 7 + c)
+    G = (torch.randn(r, c, device="cuda", generator=gen) *
+         torch.rand(1, c, device="cuda", generator=gen)).to(gdt).contiguous()
+    co = QUINTIC5[:steps]
+    # the output sits between guard bands that must stay untouched
+    band = 2048
+    store = torch.full((band + r * c + band,), -7.0, dtype=xdt, device="cuda")
+    X_na = store[band:band + r * c].view(r, c)
+    rc = f(G.data_ptr(), ns.BF16 if gdt == torch.bfloat16 else ns.FP32, X_na.data_ptr(),
+           ns.BF16 if xdt == torch.bfloat16 else ns.FP32, r, c, steps, _coeffs(ns, co) if steps else None, 1e-7,
+           status.data_ptr(), stream)
+    assert rc == ns.OK, ns.last_error()
+    X_ref = ns.ns_orthogonalize(G, steps=steps, coeffs=co if steps else None, eps=1e-7, prec="bf16",
+                                out_dtype=xdt)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0, 0]
+    assert torch.all(store[:band] == -7.0) and torch.all(store[band + r * c:] == -7.0)
+    assert torch.isfinite(X_na).all()
+    # a bf16 output adds one rounding (2^-9 relative) on top of the bf16 working precision
+    tol = TOL_O_BF16 + (4e-3 if xdt == torch.bfloat16 else 0.0)
+    assert _rel(X_na, X_ref) <= tol
+    want = ns_blas.newton_schulz(G.double().cpu().numpy(), co, eps=1e-7)
+    assert _rel(X_na.cpu(), torch.from_numpy(want)) <= tol
