@@ -235,6 +235,7 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     ns.set_wave_elements(args.wave_elements)
+    ns.set_chained_launch(args.chain)
     if world > 1:
         import torch.distributed as dist
         import datetime
@@ -348,6 +349,7 @@ def run_ours(args, world, rank, local):
                          "126 MB L2" % (elements * (4 + 4 + 2 * gbytes) / 1e9),
                    "muon_step_calls_per_step": len(call_groups),
                    "wave_elements": args.wave_elements or (1 << 29),
+                   "chained_launch": args.chain,
                    "parallelism": ("one weight set split across GPUs by Newton-Schulz FLOPs, updated parameters "
                                    "all-gathered (strong scaling)") if args.sharded else
                                   "independent weight set per GPU (weak scaling, no collective)"},
@@ -608,8 +610,11 @@ def main(argv=None):
     ap.add_argument("--step-group-layers", type=int, default=0,
                     help="device-timed step as one muon_step call per group of this many layers "
                          "(0: one call over all matrices)")
+    ap.add_argument("--no-chain", dest="chain", action="store_false",
+                    help="one launch per Newton-Schulz phase instead of one chained launch per wave of "
+                         "small matrices (see muon_set_chained_launch)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-group-layers", type=int, default=1,
                     help="layers per muon_step call in the pipelined end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")

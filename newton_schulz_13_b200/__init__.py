@@ -31,7 +31,7 @@ CUBIC = (1.5, -0.5, 0.0)
 
 EXPORTS = ["muon_ns_orthogonalize", "muon_step", "muon_adamw_step", "muon_last_error",
            "muon_check_status", "muon_release_workspace", "muon_profile_enable", "muon_profile_read",
-           "muon_launch_count", "muon_version", "muon_set_wave_elements", "muon_set_wait_limit_ns"]
+           "muon_launch_count", "muon_version", "muon_set_wave_elements", "muon_set_wait_limit_ns", "muon_set_chained_launch"]
 
 
 class MuonError(RuntimeError):
@@ -80,6 +80,8 @@ def _load() -> ctypes.CDLL:
     lib.muon_set_wave_elements.argtypes = [ctypes.c_int64]
     lib.muon_set_wait_limit_ns.restype = ctypes.c_int
     lib.muon_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.muon_set_chained_launch.restype = ctypes.c_int
+    lib.muon_set_chained_launch.argtypes = [ctypes.c_int]
     lib.muon_profile_enable.restype = ctypes.c_int
     lib.muon_profile_enable.argtypes = [ctypes.c_int]
     lib.muon_profile_read.restype = ctypes.c_int
@@ -230,6 +232,13 @@ def set_wave_elements(elements: int = 0) -> None:
     """Largest number of elements muon_step processes in one wave of launches (0: the default,
     2^29). Results do not depend on it; see muon_set_wave_elements in include/muon.h."""
     _check(lib.muon_set_wave_elements(int(elements)))
+
+
+def set_chained_launch(on: bool = True) -> None:
+    """Whole Newton-Schulz iteration of a wave of small matrices as one chained launch (default),
+    or one launch per phase. Results are bit-identical; see muon_set_chained_launch in
+    include/muon.h."""
+    _check(lib.muon_set_chained_launch(int(on)))
 
 
 def set_wait_limit_ns(ns: int = 0) -> None:

@@ -135,6 +135,10 @@ struct BufMapsX3 {   // TMA views of one two-plane fp32 buffer: K-major and MN-m
 constexpr int64_t kWaveElements = int64_t(1) << 29;
 int64_t g_wave_elements = kWaveElements;   // muon_set_wave_elements
 uint64_t g_wait_ns = 0;                     // muon_set_wait_limit_ns (0: the kernels' default)
+// Chained launches: a wave whose products all run on 256 x 256 bf16 tiles runs its whole
+// Newton-Schulz iteration (every phase of every step) as one launch (muon_set_chained_launch).
+bool g_chain = true;
+constexpr int kMaxChainPhases = 3 * MUON_MAX_NS_STEPS;
 
 // A wave: matrices [j0, j1) of the plan. Every prefix sum in the device tables (elementwise
 // chunks, column-sum items, product tiles) restarts at zero at the wave's first matrix, so a
@@ -157,6 +161,7 @@ struct Plan {
   std::vector<Shape> shapes;
   int x_bf16 = 1;
   int64_t wave_elements = 0;
+  bool chain = false;        // built for chained launches (Gram problems in matrix order)
   uint64_t arena_gen = 0;
   char* tab = nullptr;       // this plan's tables (cudaMalloc)
   size_t tab_bytes = 0;
@@ -181,6 +186,13 @@ struct Plan {
   std::vector<GemmProblem> h_upd[2][2];    // [operand: 0 B, 1 A][parity]
   std::vector<GemmProblemX3> h_upd_x3[2][2];   // the same for the fp32 (3xTF32) mode
   CUtensorMap* d_pmaps = nullptr;
+  // chained launches (bf16 waves on 256 x 256 tiles): per-matrix completion targets of the Gram,
+  // poly and update phases (eight epilogue warps per tile), the claim and completion counters,
+  // and each wave's phase list (rewritten when it changes)
+  uint32_t* d_tgt[3] = {nullptr, nullptr, nullptr};
+  uint32_t* d_chain_ctr = nullptr;
+  PhaseDesc* d_phases = nullptr;
+  std::vector<std::vector<PhaseDesc>> last_phases;   // per wave
   void* d_fused = nullptr;                 // GemmProblem (bf16) or GemmProblemX3 (fp32) table
   std::vector<uint8_t> fused_key;
 
@@ -244,13 +256,35 @@ int device_state(DeviceState** out) {
   return MUON_OK;
 }
 
+// Orders the Gram problems of each wave of small matrices (256 x 256 tiles) by descending
+// contraction length K (stable), for per-phase launches. Such a launch hands out tiles
+// round-robin over the CTA pairs in table order; a wave's Gram tiles differ in K (the longer side
+// of each matrix, up to 4x between the matrices of one model), so placing the longest tiles
+// first evens out the pairs' loads. Waves of large matrices (256 x 512 tiles, ten or more tiles
+// per pair) keep the matrix order, which measured faster there, and so do chained launches
+// (`chained`): they balance by claiming tiles as they go, and a Gram product in another order
+// than the update it waits for would start with the matrices whose updates finish last.
+template <class Prob>
+void order_gram_by_k(std::vector<Prob>& probs, const std::vector<Wave>& waves, bool chained) {
+  for (const Wave& w : waves) {
+    if (w.wide || chained) continue;
+    std::stable_sort(probs.begin() + w.j0, probs.begin() + w.j1,
+                     [](const Prob& a, const Prob& b) { return a.K > b.K; });
+    uint32_t t = 0;
+    for (int j = w.j0; j < w.j1; ++j) {
+      probs[j].tile_begin = t;
+      t += probs[j].n_tiles;
+    }
+  }
+}
+
 // Finds or builds the plan (TMA descriptors, grouped problem tables, buffer layout) of a list of
 // shapes, growing the shared buffer arena when the plan needs more than it holds.
 int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Plan** out) {
   for (size_t i = 0; i < ds.plans.size(); ++i) {
     const Plan& q = *ds.plans[i];
     if (q.shapes == shapes && q.x_bf16 == x_bf16 && q.wave_elements == g_wave_elements &&
-        q.arena_gen == ds.arena_gen) {
+        q.chain == g_chain && q.arena_gen == ds.arena_gen) {
       if (i > 0) std::rotate(ds.plans.begin(), ds.plans.begin() + i, ds.plans.begin() + i + 1);
       *out = ds.plans[0].get();
       return MUON_OK;
@@ -260,6 +294,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   P->shapes = shapes;
   P->x_bf16 = x_bf16;
   P->wave_elements = g_wave_elements;
+  P->chain = g_chain;
   const int n = (int)shapes.size();
   // bf16 mode: one bf16 plane per buffer; fp32 mode: hi and lo fp32 planes (GemmProblemX3)
   const size_t esz = x_bf16 ? 2 : 8;
@@ -355,6 +390,12 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   if (x_bf16) off = align_up(off + (size_t)n * sizeof(CUtensorMap), AL);
   const size_t o_fused = off;
   off = align_up(off + (size_t)n * prob_sz, AL);
+  const size_t o_tgt = off;
+  off = align_up(off + 3 * (size_t)n * 4, AL);
+  const size_t o_ctr = off;
+  off = align_up(off + (1 + (size_t)kMaxChainPhases * n) * 4, AL);
+  const size_t o_phases = off;
+  off = align_up(off + P->waves.size() * (size_t)kMaxChainPhases * sizeof(PhaseDesc), AL);
   P->tab_bytes = off;
 
   auto alloc_fail = [](cudaError_t e, const char* what, size_t bytes) {
@@ -388,6 +429,10 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   char* T = P->tab;     // tables
   P->d_partials = reinterpret_cast<float*>(W + o_part);
   P->d_mats = reinterpret_cast<MatInfo*>(T + o_mats);
+  for (int k = 0; k < 3; ++k) P->d_tgt[k] = reinterpret_cast<uint32_t*>(T + o_tgt) + (size_t)k * n;
+  P->d_chain_ctr = reinterpret_cast<uint32_t*>(T + o_ctr);
+  P->d_phases = reinterpret_cast<PhaseDesc*>(T + o_phases);
+  P->last_phases.assign(P->waves.size(), {});
   for (int j = 0; j < n; ++j) {
     P->x0.push_back(W + o_x0[j]);
     P->x1.push_back(W + o_x1[j]);
@@ -465,25 +510,32 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
         g.K = (uint32_t)nn;
         g.tiles_m = (uint32_t)ceil_div(m, kTcPairBM);
         g.tiles_n = (uint32_t)ceil_div(m, w.wide ? kTcWideBN : kTcBN);
-        g.sym = 1;
+        g.sym = w.wide ? 1 : 2;   // A whole (mirrored writes) or in the upper-block form
+        g.mat = (uint16_t)j;
         g.n_tiles = (uint32_t)(w.wide ? sym_tiles_wide(m) : sym_tiles(m));
         g.tile_begin = tg;
         gram[p].push_back(g);
         for (int which = 0; which < 2; ++which) {   // 0: operand B, 1: operand A
           const BufMaps& mS = which == 0 ? mB : mA;
           GemmProblem u{};
+          // B (or A) in the upper-block form: K slices below its diagonal blocks are read
+          // transposed through its MN-major view
+          const uint8_t half = w.wide ? 0 : 1;
           if (!tall) {
             u.tma_a = M_(mS.k128); u.a_mn = 0;
+            u.tma_a_t = M_(mS.mn64); u.a_half = half;
             u.tma_b = M_(mx[p].mn64); u.b_mn = 1;
           } else {
             u.tma_a = M_(mx[p].k128); u.a_mn = 0;
             u.tma_b = M_(mS.k128); u.b_mn = 0;
+            u.tma_b_t = M_(mS.mn64); u.b_half = half;
           }
           u.d = static_cast<__nv_bfloat16*>(p == 0 ? P->x1[j] : P->x0[j]);
           u.ldd = P->ldx[j];
           u.tma_d = M_(mx[1 - p].st32);
           u.alpha = P->alpha[j];
           u.M = (uint32_t)r; u.N = (uint32_t)c; u.K = (uint32_t)m;
+          u.mat = (uint16_t)j;
           u.tiles_m = (uint32_t)ceil_div(r, kTcPairBM);
           u.tiles_n = (uint32_t)ceil_div(c, w.wide ? kTcWideBN : kTcBN);
           u.n_tiles = u.tiles_m * u.tiles_n;
@@ -492,8 +544,12 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
         }
       }
       GemmProblem q{};
-      // B = c A A + b A (+ a I on the tensor-core path): A is symmetric, so A A = A A^T
+      // B = c A A + b A (+ a I on the tensor-core path): A is symmetric, so A A = A A^T; A and B
+      // are in the upper-block form
       q.tma_a = M_(mA.k128); q.tma_b = M_(mA.k128);
+      q.tma_a_t = M_(mA.mn64); q.tma_b_t = M_(mA.mn64);
+      q.a_half = q.b_half = w.wide ? 0 : 1;
+      q.mat = (uint16_t)j;
       q.d = static_cast<__nv_bfloat16*>(P->B[j]); q.ldd = P->ldm[j];
       q.tma_d = M_(mB.st32);
       q.tma_c = M_(mA.st32);
@@ -501,7 +557,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       q.M = q.N = q.K = (uint32_t)m;
       // the polynomial product (K = m) stays on 256 x 256 tiles: its triangle wastes less there
       q.tiles_m = (uint32_t)ceil_div(m, kTcPairBM); q.tiles_n = (uint32_t)ceil_div(m, kTcBN);
-      q.sym = 1;
+      q.sym = w.wide ? 1 : 2;
       q.n_tiles = (uint32_t)sym_tiles(m);
       q.tile_begin = tp;
       poly.push_back(q);
@@ -519,6 +575,18 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     }
     if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
     MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+    {
+      // completion targets of a chained launch: eight epilogue warps per tile of each matrix
+      std::vector<uint32_t> tgt(3 * (size_t)n);
+      for (int j = 0; j < n; ++j) {
+        tgt[j] = 8u * gram[0][j].n_tiles;
+        tgt[n + j] = 8u * poly[j].n_tiles;
+        tgt[2 * (size_t)n + j] = 8u * updB[0][j].n_tiles;
+      }
+      MUON_CUDA(cudaMemcpy(P->d_tgt[0], tgt.data(), tgt.size() * 4, cudaMemcpyHostToDevice));
+    }
+    order_gram_by_k(gram[0], P->waves, P->chain);
+    order_gram_by_k(gram[1], P->waves, P->chain);
     std::vector<GemmProblem>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
                       &P->d_updA[0], &P->d_updA[1]};
@@ -633,6 +701,8 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     }
     if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
     MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
+    order_gram_by_k(gram[0], P->waves, false);
+    order_gram_by_k(gram[1], P->waves, false);
     std::vector<GemmProblemX3>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
                       &P->d_updA[0], &P->d_updA[1]};
@@ -763,11 +833,88 @@ int check_shape(int64_t r, int64_t c, const char* what) {
   return MUON_OK;
 }
 
-// Runs the Newton-Schulz phases for the matrices of one wave. fused_last (optional) is the
-// per-call table of last-update problems for all matrices of the plan.
-int run_ns(DeviceState& ds, Plan& P, const Wave& w, const std::vector<muon_coeffs_t>& co, cudaStream_t s,
-           const void* fused_last = nullptr, float lr = 0.0f, float decay = 1.0f) {
+// The whole Newton-Schulz iteration of one wave as one chained launch (bf16, 256 x 256 tiles):
+// the same phases, problem tables and epilogue scalars as the per-phase launches of run_ns, with
+// each phase waiting (per matrix) for the one whose results it reads: Gram k for update k - 1,
+// poly k for Gram k, update k for poly k (Gram k when c_k = 0).
+int run_ns_chained(DeviceState& ds, Plan& P, const Wave& w, int wave_idx, const std::vector<muon_coeffs_t>& co,
+                   cudaStream_t s, const void* fused_last, float lr, float decay) {
   const int n = w.j1 - w.j0;
+  auto tc = [&](void* t) { return static_cast<GemmProblem*>(t) + w.j0; };
+  std::vector<PhaseDesc> ph;
+  uint32_t tiles = 0;
+  double fl = 0.0, ex = 0.0;
+  auto add = [&](const void* table, uint32_t n_tiles, const EpiScalars& e, int dep, const uint32_t* tgt) {
+    PhaseDesc d{};
+    d.probs = static_cast<const GemmProblem*>(table);
+    d.dep_target = dep >= 0 ? tgt : nullptr;
+    d.tile_begin = tiles;
+    d.nprobs = n;
+    d.dep = dep;
+    d.ep = e;
+    d.ep.wait_ns = g_wait_ns;
+    ph.push_back(d);
+    tiles += n_tiles;
+    return (int)ph.size() - 1;
+  };
+  int prev_update = -1;
+  for (size_t k = 0; k < co.size(); ++k) {
+    const int p = (int)(k & 1);
+    const int first = k == 0 ? 1 : 0;
+    const muon_coeffs_t c = co[k];
+    // the same epilogue scalars as run_ns's bf16 path
+    EpiScalars eg{1.0f, 0.0f, first ? 2 : 0, 0, 0.0f};
+    if (c.c == 0.0f) eg = EpiScalars{c.b, 0.0f, first ? 2 : 0, 0, c.a};
+    const int gram = add(tc(P.d_gram[p]), w.tiles_gram, eg, prev_update, P.d_tgt[2]);
+    fl += w.fl_gram;
+    ex += w.ex_gram;
+    int dep = gram;
+    const uint32_t* dep_tgt = P.d_tgt[0];
+    void* upd = P.d_updA[p];
+    if (c.c != 0.0f) {
+      dep = add(tc(P.d_poly), w.tiles_poly, EpiScalars{c.c, c.b, 0, 0, c.a}, gram, P.d_tgt[0]);
+      dep_tgt = P.d_tgt[1];
+      upd = P.d_updB[p];
+      fl += w.fl_poly;
+      ex += w.ex_poly;
+    }
+    EpiScalars eu{1.0f, 0.0f, first, 0, 0.0f};
+    if (fused_last && k + 1 == co.size()) {
+      upd = const_cast<void*>(fused_last);
+      eu.lr = lr;
+      eu.decay = decay;
+      eu.fused = 1;
+    }
+    prev_update = add(tc(upd), w.tiles_upd, eu, dep, dep_tgt);
+    fl += w.fl_upd;
+    ex += w.ex_upd;
+  }
+  PhaseDesc* d_ph = P.d_phases + (size_t)wave_idx * kMaxChainPhases;
+  std::vector<PhaseDesc>& last = P.last_phases[wave_idx];
+  if (last.size() != ph.size() || std::memcmp(last.data(), ph.data(), ph.size() * sizeof(PhaseDesc)) != 0) {
+    MUON_CUDA(write_table(d_ph, ph.data(), ph.size() * sizeof(PhaseDesc), s, &g_launches));
+    last = ph;
+  }
+  const int nmats = (int)P.shapes.size();
+  MUON_CUDA(cudaMemsetAsync(P.d_chain_ctr, 0, (1 + ph.size() * (size_t)nmats) * 4, s));
+  const ChainArgs ca{d_ph, P.d_chain_ctr, P.d_chain_ctr + 1, (int)ph.size(), nmats};
+  EpiScalars el{};
+  el.wait_ns = g_wait_ns;
+  cudaError_t e = timed_launch(MUON_KC_GEMM, s, fl, ex, [&] {
+    return launch_gemm_tc_pair_chain(ca, tiles, el, ds.d_status, ds.pair_capacity, s);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "chained Newton-Schulz launch");
+  return MUON_OK;
+}
+
+// Runs the Newton-Schulz phases for the matrices of one wave (wave_idx of the plan). fused_last
+// (optional) is the per-call table of last-update problems for all matrices of the plan.
+int run_ns(DeviceState& ds, Plan& P, const Wave& w, int wave_idx, const std::vector<muon_coeffs_t>& co,
+           cudaStream_t s, const void* fused_last = nullptr, float lr = 0.0f, float decay = 1.0f) {
+  const int n = w.j1 - w.j0;
+  if (P.x_bf16 && !w.wide && g_chain && !co.empty() && co.size() * 3 <= (size_t)kMaxChainPhases &&
+      P.shapes.size() <= 65535)
+    return run_ns_chained(ds, P, w, wave_idx, co, s, fused_last, lr, decay);
   // the wave's sub-range of a problem table
   auto tc = [&](void* t) { return static_cast<GemmProblem*>(t) + w.j0; };
   auto x3 = [&](void* t) { return static_cast<GemmProblemX3*>(t) + w.j0; };
@@ -949,6 +1096,13 @@ int muon_set_wave_elements(int64_t elements) {
   return MUON_OK;
 }
 
+int muon_set_chained_launch(int on) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  t_err.clear();
+  g_chain = on != 0;
+  return MUON_OK;
+}
+
 int muon_set_wait_limit_ns(uint64_t ns) {
   std::lock_guard<std::mutex> lk(g_mu);
   t_err.clear();
@@ -1033,7 +1187,8 @@ int muon_step(int count, float* const* params, const void* const* grads, muon_dt
   }
 
   const int ew_grid = ds->sms * 8;
-  for (const Wave& w : P->waves) {
+  for (size_t wi = 0; wi < P->waves.size(); ++wi) {
+    const Wave& w = P->waves[wi];
     const MatInfo* dm = P->d_mats + w.j0;
     const int nw = w.j1 - w.j0;
     cudaError_t e;
@@ -1050,7 +1205,7 @@ int muon_step(int count, float* const* params, const void* const* grads, muon_dt
     if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
     e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(dm, nw, P->d_partials, eps, s); });
     if (e != cudaSuccess) return cuda_fail(e, "norm launch");
-    rc = run_ns(*ds, *P, w, co, s, fused, lr, 1.0f - lr * weight_decay);
+    rc = run_ns(*ds, *P, w, (int)wi, co, s, fused, lr, 1.0f - lr * weight_decay);
     if (rc != MUON_OK) return rc;
     if (fused) continue;   // the last update product already wrote the parameters
     e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
@@ -1200,7 +1355,7 @@ int muon_ns_orthogonalize(const void* G, muon_dtype_t g_dtype, void* X, muon_dty
   if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
   e = timed_launch(MUON_KC_NORM, s, 0, 0, [&] { return launch_alpha(P->d_mats, 1, P->d_partials, eps, s); });
   if (e != cudaSuccess) return cuda_fail(e, "norm launch");
-  rc = run_ns(*ds, *P, w, co, s);
+  rc = run_ns(*ds, *P, w, 0, co, s);
   if (rc != MUON_OK) return rc;
   e = timed_launch(MUON_KC_EPILOGUE, s, 0, 0, [&] {
     return launch_output(P->d_mats, 1, w.n_chunks, x_bf16, x_dtype == MUON_BF16, steps == 0 ? 1 : 0,

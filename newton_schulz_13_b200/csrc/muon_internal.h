@@ -65,6 +65,10 @@ struct AdamScalars {
 struct GemmProblem {
   const CUtensorMap* tma_a;
   const CUtensorMap* tma_b;
+  // CTA-pair kernel, a_half / b_half operands: the MN-major view of the same matrix, for the K
+  // slices read transposed (see a_half below)
+  const CUtensorMap* tma_a_t;
+  const CUtensorMap* tma_b_t;
   const CUtensorMap* tma_d;   // CTA-pair kernel: TMA store view (32 x 32 boxes) of d
   const CUtensorMap* tma_c;   // CTA-pair kernel: TMA load view (32 x 32 boxes) of the addend, or NULL
   const CUtensorMap* tma_p;   // CTA-pair kernel, fused last update: fp32 parameters (32 x 32 boxes)
@@ -78,9 +82,15 @@ struct GemmProblem {
   uint32_t n_tiles;
   float rms;                // fused last update: RMS factor s of this matrix
   uint8_t a_mn, b_mn;       // 1: operand is MN-major
-  uint8_t sym;              // 1: D is symmetric, compute tiles touching the upper triangle
-                            //    and write the strictly-upper part mirrored
+  uint8_t sym;              // D is symmetric: compute the tiles touching the upper triangle, and
+                            //   1: write the strictly-upper part also mirrored (whole matrix);
+                            //   2 (CTA-pair kernel): write only the 256 x 256 blocks on or above
+                            //      the diagonal (the upper-block form)
+  uint8_t a_half, b_half;   // 1 (CTA-pair kernel): the operand is a symmetric matrix in the
+                            //   upper-block form; a K slice in a 256-block below the operand rows'
+                            //   block is read transposed, from the mirror block, through tma_*_t
   uint8_t pad;
+  uint16_t mat;             // chained launch: the problem's matrix (index within its plan)
 };
 
 // fp32 precision mode ("3xTF32"). Every fp32 matrix of the iteration is held as two planes of
@@ -124,6 +134,30 @@ struct EpiScalars {
   uint64_t wait_ns;
 };
 
+// Chained launch (CTA-pair kernel, 256 x 256 tiles): one launch runs every Newton-Schulz product
+// of a wave, phase after phase. Global tile t belongs to the phase with the largest
+// tile_begin <= t; its tiles are that phase's problem table, scheduled as in a launch of its own.
+// A tile of a phase with a dependency reads results of the phase `dep` for the same matrix: it
+// starts once done[dep][mat] (epilogue warps that finished a tile of that matrix, eight per tile)
+// has reached dep_target[mat].
+struct PhaseDesc {
+  const GemmProblem* probs;
+  const uint32_t* dep_target;   // per matrix of the plan, or NULL when dep < 0
+  uint32_t tile_begin;
+  int nprobs;
+  int dep;
+  int pad;
+  EpiScalars ep;
+};
+
+struct ChainArgs {
+  const PhaseDesc* phases;
+  uint32_t* tile_counter;   // tiles claimed so far (zero before the launch)
+  uint32_t* done;           // [phase][matrix] finished epilogue warps (zero before the launch)
+  int nphases;
+  int nmats;                // matrices of the plan (the row length of done)
+};
+
 // Per-call tables (pointer tables of a call) travel to the device inside kernel parameters, not
 // through a copy engine: a small copy on the caller's stream would otherwise queue behind whatever
 // bulk copies the caller has in flight (up to the whole step's gradient upload).
@@ -158,6 +192,10 @@ cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t t
 // The same with 256 x kTcWideBN tiles (problem tables built with tiles_n = ceil(N / kTcWideBN)).
 cudaError_t launch_gemm_tc_pair_wide(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                      EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
+// Every phase of a wave in one launch (256 x 256 tiles); fa's counters must be zero. ep carries
+// only the launch's wait limit.
+cudaError_t launch_gemm_tc_pair_chain(ChainArgs fa, uint32_t total_tiles, EpiScalars ep, int* status,
+                                      int max_pairs, cudaStream_t s);
 int gemm_tc_pair_capacity(int sms);
 cudaError_t launch_gemm_x3(const GemmProblemX3* probs, int nprobs, uint32_t total_tiles,
                            EpiScalars ep, int* status, int max_pairs, cudaStream_t s);

@@ -75,15 +75,24 @@ struct TcCfg {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kEpiArrivals = PAIR ? 8 : 4;
-  // CTA pair: per epilogue warp two staging sets (direct + mirrored 32 x 32 bf16 sub-tiles)
-  static constexpr uint32_t kStagingPerWarp = 2 * 2 * 2048;
+  // CTA pair: 8 KB of staging per epilogue warp (four 32 x 32 bf16 sub-tiles, or two fp32 ones)
+  static constexpr uint32_t kStagingPerWarp = 4 * 2048;
   static constexpr uint32_t kStagingBytes = PAIR ? 4 * kStagingPerWarp : 0;
-  static constexpr size_t kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 256;
-  // the 256-byte tail: full and empty per stage, tfull and tempty per accumulator, drain and 8
-  // epilogue load barriers; then the tensor-memory address, two flags and the producer's fill count
-  static_assert((2 * kStages + 2 + 2 + 9) * 8 + 4 * 4 <= 256, "barrier area");
+  static constexpr size_t kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 512;
+  // the 512-byte tail: full and empty per stage, tfull and tempty per accumulator, drain, 16
+  // epilogue operand-load barriers (4 per epilogue warp) and the tile queue's 2 x 8 barriers; then
+  // the tensor-memory address, two flags, the producer's fill count and the 8 queued tiles
+  static_assert((2 * kStages + 2 + 2 + 33) * 8 + 12 * 4 <= 512, "barrier area");
   static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA");
 };
+
+// Whether K slice kb of an operand is read MN-major: always for an MN-major operand; for a
+// symmetric operand in the upper-block form (half), when the slice's 256-block of K lies below the
+// 256-block `rblk` of the operand's rows, where only the mirror block (K rows, operand columns) is
+// stored. Both CTAs of a pair and every 16-deep MMA of a slice make the same choice.
+__device__ __forceinline__ bool slice_mn(uint8_t mn, uint8_t half, uint32_t kb, uint32_t rblk) {
+  return mn || (half && (kb * (uint32_t)kTcBK) / 256u < rblk);
+}
 
 // Byte offset of 16-byte chunk j of row r in a 32-row x 64-byte staging box laid out with the
 // 64-byte swizzle the TMA store expects (chunk index XOR bits 1-2 of the row).
@@ -91,10 +100,23 @@ __device__ __forceinline__ uint32_t sw64_chunk(uint32_t r, uint32_t j) {
   return r * 64u + ((j ^ ((r >> 1) & 3u)) << 4);
 }
 
-template <bool PAIR, bool WIDE>
+// Chained launches: the tile queue's depth, and the roles that read each queued tile (the MMA
+// thread, the odd CTA's producer and the eight epilogue warps of the pair).
+constexpr int kTileQ = 8;
+constexpr uint32_t kTileQReaders = 10;
+constexpr uint32_t kNoTile = 0xffffffffu;
+
+// CHAIN (CTA pair, 256 x 256 tiles): the launch runs all the phases of ca (see PhaseDesc). Tiles
+// are claimed in order, with an atomic add, by the even CTA's producer and handed to the pair's
+// other roles through a queue in shared memory; a tile waits for the phase it reads (per
+// matrix) before its operands are loaded, and each epilogue warp counts its finished tiles. A
+// claimed tile depends only on tiles claimed before it, so the launch makes progress whether or
+// not all of its CTAs are resident.
+template <bool PAIR, bool WIDE, bool CHAIN>
 __global__ void __launch_bounds__(kThreads, 1)
     ns_gemm_tc_kernel(const GemmProblem* __restrict__ probs, int nprobs, uint32_t total_tiles,
-                      EpiScalars ep, int* __restrict__ status) {
+                      EpiScalars ep, int* __restrict__ status, ChainArgs ca) {
+  static_assert(!CHAIN || (PAIR && !WIDE), "chained launches use 256 x 256 CTA-pair tiles");
   using C = TcCfg<PAIR, WIDE>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -104,11 +126,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;                       // followed by 8 operand-load barriers
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 9);
+  uint64_t* drain = tempty + 2;                       // followed by 16 operand-load barriers
+  uint64_t* tq_full = drain + 17;                     // tile queue (chained launches)
+  uint64_t* tq_empty = tq_full + kTileQ;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kTileQ);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* zero_flag = abort_flag + 1;   // never set: the drain waits poll it
   volatile uint32_t* fill_count = reinterpret_cast<volatile uint32_t*>(zero_flag + 1);
+  volatile uint32_t* tq = fill_count + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = PAIR ? cluster_ctarank() : 0u;      // 0: the CTA that issues the MMAs
@@ -127,7 +152,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tempty[a], C::kEpiArrivals);
     }
     mbar_init(drain, 1);
-    for (int w = 0; w < 8; ++w) mbar_init(drain + 1 + w, 1);
+    for (int w = 0; w < 16; ++w) mbar_init(drain + 1 + w, 1);
+    for (int q = 0; q < kTileQ; ++q) {
+      mbar_init(&tq_full[q], 1);
+      mbar_init(&tq_empty[q], kTileQReaders);
+    }
     *abort_flag = 0;
     *zero_flag = 0;
     *fill_count = 0;
@@ -150,19 +179,102 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   bool timed_out = false;
 
+  // ---- the tiles of this CTA (pair), in order. seq counts the tiles a role has taken; returns
+  // false when there are no more (or a wait gave up, and timed_out is set). Static launches walk
+  // the tile index with a stride of n_units. Chained launches: the even CTA's producer (claimer)
+  // takes the next index with an atomic add and queues it in both CTAs; the other roles read it
+  // from their CTA's queue (warp_wide: every lane of an epilogue warp) and release the entry.
+  auto next_tile = [&](uint32_t& seq, uint32_t& t, bool claimer, bool warp_wide) -> bool {
+    if constexpr (!CHAIN) {
+      t = unit + seq * n_units;
+      ++seq;
+      return t < total_tiles;
+    } else {
+      const uint32_t q = seq % kTileQ, par = (seq / kTileQ) & 1u;
+      if (claimer) {
+        if (!mbar_wait_bounded(&tq_empty[q], par ^ 1u, abort_flag, wait_ns)) {
+          timed_out = true;
+          return false;
+        }
+        uint32_t v = atomicAdd(ca.tile_counter, 1u);
+        if (v >= total_tiles) v = kNoTile;
+        tq[q] = v;
+        st_shared_cluster(mapa_shared(smem_u32((const void*)&tq[q]), 1u), v);
+        mbar_arrive(&tq_full[q]);
+        mbar_arrive_cluster(mapa_shared(smem_u32(&tq_full[q]), 1u));
+        t = v;
+      } else {
+        bool ok = mbar_wait_cluster_bounded(&tq_full[q], par, abort_flag, wait_ns);
+        if (warp_wide) ok = __all_sync(0xffffffffu, ok);
+        if (!ok) {
+          timed_out = true;
+          return false;
+        }
+        t = tq[q];
+        if (!warp_wide || lane == 0) {
+          if (leader) mbar_arrive(&tq_empty[q]);
+          else mbar_arrive_cluster(mapa_shared(smem_u32(&tq_empty[q]), 0u));
+        }
+      }
+      ++seq;
+      return t != kNoTile;
+    }
+  };
+  // problem, tile coordinates, epilogue scalars and phase of global tile t
+  auto decode = [&](uint32_t t, Tile& tl, const GemmProblem*& P, const EpiScalars*& E, int& ph) {
+    if constexpr (CHAIN) {
+      int lo = 0, hi = ca.nphases - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (ca.phases[mid].tile_begin <= t) lo = mid; else hi = mid - 1;
+      }
+      const PhaseDesc& D = ca.phases[lo];
+      tl = decode_tile<C::kTileM, C::kTileN>(D.probs, D.nprobs, t - D.tile_begin);
+      P = &D.probs[tl.p];
+      E = &D.ep;
+      ph = lo;
+    } else {
+      tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
+      P = &probs[tl.p];
+      E = &ep;
+      ph = 0;
+    }
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (every CTA)
     if (lane == 0) {
       int issued_parity[C::kStages];
       for (int s = 0; s < C::kStages; ++s) issued_parity[s] = -1;
-      uint32_t stage = 0, phase = 0, fills = 0;
-      for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
-        const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
-        const GemmProblem& P = probs[tl.p];
+      uint32_t stage = 0, phase = 0, fills = 0, seq = 0, t = 0;
+      while (!timed_out && next_tile(seq, t, leader, false)) {
+        Tile tl;
+        const GemmProblem* Pp;
+        const EpiScalars* Ep;
+        int ph;
+        decode(t, tl, Pp, Ep, ph);
+        // a copy in registers: the asm statements below clobber memory, which would make every use
+        // of a field of the table in global memory a fresh load
+        const GemmProblem P = *Pp;
+        if constexpr (CHAIN) {
+          // the results this tile reads (same matrix, earlier phase) must be complete
+          const PhaseDesc& D = ca.phases[ph];
+          if (D.dep >= 0) {
+            if (!counter_wait_bounded(ca.done + (size_t)D.dep * ca.nmats + P.mat, D.dep_target[P.mat], abort_flag,
+                                      wait_ns)) {
+              timed_out = true;
+              break;
+            }
+            fence_proxy_async_global();
+          }
+        }
         const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
         const int32_t a_row0 = (int32_t)(tl.bi * C::kTileM + rank * 128);
         // single CTA: all 256 opB rows of the tile; pair: this CTA's 128 rows of each 256-wide half
         const int32_t b_row0 = (int32_t)(tl.bj * C::kTileN + rank * (PAIR ? 128 : 0));
+        // 256-blocks of the operands' rows (symmetric operands in the upper-block form)
+        const uint32_t rblk_a = (tl.bi * C::kTileM) / 256u;
+        auto rblk_b = [&](int hf) { return (tl.bj * C::kTileN + 256u * (uint32_t)hf) / 256u; };
         for (uint32_t kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, wait_ns)) {
             timed_out = true;
@@ -175,21 +287,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             // both halves of the pair count on the even CTA's barrier
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
-            if (!P.a_mn) {
+            if (!slice_mn(P.a_mn, P.a_half, kb, rblk_a)) {
               tma_load_2d_pair(a_dst, P.tma_a, bar, k0, a_row0);
             } else {
+              const CUtensorMap* map = P.a_mn ? P.tma_a : P.tma_a_t;
               for (int h = 0; h < 2; ++h)
-                tma_load_2d_pair(a_dst + h * kBoxBytes, P.tma_a, bar, a_row0 + 64 * h, k0);
+                tma_load_2d_pair(a_dst + h * kBoxBytes, map, bar, a_row0 + 64 * h, k0);
             }
 #pragma unroll
             for (int hf = 0; hf < C::kHalves; ++hf) {
               uint8_t* bh = b_dst + hf * C::kBHalfBytes;
               const int32_t brow = b_row0 + 256 * hf;
-              if (!P.b_mn) {
+              if (!slice_mn(P.b_mn, P.b_half, kb, rblk_b(hf))) {
                 tma_load_2d_pair(bh, P.tma_b, bar, k0, brow);
               } else {
+                const CUtensorMap* map = P.b_mn ? P.tma_b : P.tma_b_t;
                 for (int h = 0; h < 2; ++h)
-                  tma_load_2d_pair(bh + h * kBoxBytes, P.tma_b, bar, brow + 64 * h, k0);
+                  tma_load_2d_pair(bh + h * kBoxBytes, map, bar, brow + 64 * h, k0);
               }
             }
           } else {
@@ -226,17 +340,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && leader) {
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
-      for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
-        const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
-        const GemmProblem& P = probs[tl.p];
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, seq = 0, t = 0;
+      while (!timed_out && next_tile(seq, t, false, false)) {
+        Tile tl;
+        const GemmProblem* Pp;
+        const EpiScalars* Ep;
+        int ph;
+        decode(t, tl, Pp, Ep, ph);
+        const GemmProblem P = *Pp;   // in registers (see the producer)
         const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
-        // every MMA is kTileM x 256 x 16 (the wide tile issues one per half)
-        const uint32_t idesc = idesc_bf16_f32(C::kTileM, 256, P.a_mn, P.b_mn);
-        const uint32_t a_lbo = P.a_mn ? kBoxBytes : 16u, b_lbo = P.b_mn ? kBoxBytes : 16u;
-        const uint32_t a_kstep = P.a_mn ? 16u * 128u : 32u, b_kstep = P.b_mn ? 16u * 128u : 32u;
-        // the MMAs of one K slice (64 deep) for one 256-column half
-        auto issue = [&](uint32_t stg, int hf, bool first_slice) {
+        const uint32_t rblk_a = (tl.bi * C::kTileM) / 256u;
+        // the MMAs (kTileM x 256 x 16 each; the wide tile issues them per half) of K slice kb for
+        // one 256-column half; the operand layouts follow the producer's choice for that slice
+        auto issue = [&](uint32_t stg, int hf, bool first_slice, uint32_t kb) {
+          const uint32_t amn = slice_mn(P.a_mn, P.a_half, kb, rblk_a) ? 1u : 0u;
+          const uint32_t bmn = slice_mn(P.b_mn, P.b_half, kb, (tl.bj * C::kTileN + 256u * (uint32_t)hf) / 256u) ? 1u : 0u;
+          const uint32_t idesc = idesc_bf16_f32(C::kTileM, 256, amn, bmn);
+          const uint32_t a_lbo = amn ? kBoxBytes : 16u, b_lbo = bmn ? kBoxBytes : 16u;
+          const uint32_t a_kstep = amn ? 16u * 128u : 32u, b_kstep = bmn ? 16u * 128u : 32u;
           const uint32_t a_addr = smem_u32(smem + stg * C::kStageBytes);
           const uint32_t b_addr = a_addr + C::kABytes + hf * C::kBHalfBytes;
           const uint32_t d_tmem = tmem_base + (WIDE ? hf : acc) * 256u;
@@ -265,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            issue(stage, 0, kb == 0);
+            issue(stage, 0, kb == 0, kb);
             release(stage);
             if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
@@ -290,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            issue(st, 0, i == 0);
+            issue(st, 0, i == 0, i);
             if (++st == C::kStages) { st = 0; ph ^= 1u; }
           }
           if (timed_out) break;
@@ -300,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           for (uint32_t i = 0; i < npre; ++i) {
-            issue(stage, 1, i == 0);
+            issue(stage, 1, i == 0, i);
             release(stage);
             if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
@@ -310,8 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            issue(stage, 0, false);
-            issue(stage, 1, false);
+            issue(stage, 0, false, kb);
+            issue(stage, 1, false, kb);
             release(stage);
             if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
@@ -332,24 +453,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Each warp owns 32 accumulator rows. Per 32-column chunk it forms
     //   D = k_acc alpha^e acc + k_c C + diag I
     // in fp32, rounds to bf16, stages the 32 x 32 sub-tile in shared memory (64-byte swizzle) and
-    // writes it with a TMA store. The addend sub-tile C, when there is one, arrives by TMA in the
-    // same staging buffer first. For symmetric outputs, sub-tiles strictly above the diagonal are
-    // also staged transposed and stored at the mirrored position, sub-tiles strictly below are
-    // skipped (their mirror writes them) and diagonal sub-tiles are stored whole. Rows and
-    // columns past the matrix are clipped by the TMA store.
-    // Sub-tiles alternate between two staging sets. When the epilogue reads an operand sub-tile
-    // (the addend, or the parameters of the fused update), the load of the tile's next active
-    // sub-tile goes out into the other set before this one's arithmetic, so its latency overlaps.
+    // writes it with a TMA store; rows and columns past the matrix are clipped by the store. A
+    // symmetric output is written whole (sym 1: sub-tiles strictly above the diagonal are also
+    // staged transposed and stored at the mirrored position, those strictly below are skipped)
+    // or in the upper-block form (sym 2: chunks in a 256-block below the diagonal are skipped).
+    // The chunks a tile writes ("active") are one contiguous range.
+    // Staging is a ring of slots per warp (8 KB) that the active chunks use in turn: four 2 KB
+    // slots (bf16 sub-tiles), or two 4 KB slots for the fused last update (fp32 parameter
+    // sub-tiles) and for whole symmetric outputs (a sub-tile and its mirror). A chunk that reads an
+    // operand sub-tile (the addend C, or the parameters) has its load issued `ahead` active chunks
+    // earlier (2 with 2 KB slots, 1 with 4 KB slots) into the slot it will use, once the store
+    // that used that slot last has read it.
     const uint32_t quarter = (uint32_t)(warp & 3);
     uint8_t* stg = staging + (uint32_t)(warp - 2) * C::kStagingPerWarp;
-    uint64_t* cbar = drain + 1 + 2 * (warp - 2);   // this warp's operand-load barriers, one per set
-    uint32_t set = 0, cph = 0;                     // cph bit s: phase of cbar[s]
-    uint32_t inflight = 0;                         // bit s: a load into set s not yet waited for
-    int pend = -1;                                 // sub-tile whose load was issued ahead
-    uint32_t acc = 0, acc_phase = 0;
-    for (uint32_t t = unit; t < total_tiles; t += n_units) {
-      const Tile tl = decode_tile<C::kTileM, C::kTileN>(probs, nprobs, t);
-      const GemmProblem& P = probs[tl.p];
+    uint64_t* cbar = drain + 1 + 4 * (warp - 2);   // this warp's operand-load barriers, one per slot
+    uint32_t cph = 0;        // bit s: phase of cbar[s]
+    uint32_t inflight = 0;   // bit s: a load into slot s not yet waited for
+    uint32_t ring = 0;       // slot of the next active chunk
+    int geo = -1;            // slot geometry in use: 0 four 2 KB slots, 1 two 4 KB slots
+    uint32_t acc = 0, acc_phase = 0, seq = 0, t = 0;
+    while (next_tile(seq, t, false, true)) {
+      Tile tl;
+      const GemmProblem* Pp;
+      const EpiScalars* Ep;
+      int ph;
+      decode(t, tl, Pp, Ep, ph);
+      const GemmProblem P = *Pp;   // in registers (see the producer)
+      const EpiScalars ep = *Ep;   // this tile's phase (the launch's own scalars when not chained)
       const float alpha = ep.e_acc ? *P.alpha : 1.0f;
       const float s1 = ep.k_acc * alpha_pow(alpha, ep.e_acc);
       const bool has_c = P.tma_c != nullptr && ep.k_c != 0.0f;
@@ -362,27 +492,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int32_t r0 = (int32_t)(tl.bi * C::kTileM + rank * 128 + quarter * 32);
-      // sub-tiles that produce output (the same for every lane)
-      auto active = [&](int c) {
-        const int32_t cc = (int32_t)(tl.bj * C::kTileN + c * 32);
-        return r0 < (int32_t)P.M && cc < (int32_t)P.N && !(P.sym && cc + 32 <= r0);
+      const int32_t col0 = (int32_t)(tl.bj * C::kTileN);
+      const bool fused = ep.fused != 0;
+      const bool whole_sym = P.sym == 1;
+      const int g = (fused || whole_sym) ? 1 : 0;
+      if (g != geo) {   // the slots change size: every earlier store has read its slot
+        if (lane == 0) bulk_wait_group_read<0>();
+        __syncwarp();
+        ring = 0;
+        geo = g;
+      }
+      const uint32_t nslot = g ? 2u : 4u, slot_bytes = g ? 4096u : 2048u;
+      const int ahead = g ? 1 : 2;
+      // active chunks [lo, hi): inside the matrix and, for a symmetric output, not below the
+      // 32 x 32 diagonal (whole form) or in a 256-block on or above the diagonal (upper-block
+      // form); the same for every lane
+      int lo = 0, hi = 0;
+      if (r0 < (int32_t)P.M && col0 < (int32_t)P.N) {
+        hi = min(C::kTileN / 32, ((int32_t)P.N - col0 + 31) / 32);
+        const int32_t first = whole_sym ? r0 : (P.sym ? (int32_t)(tl.bi * C::kTileM) : col0);
+        lo = min(hi, max(0, (first - col0) / 32));
+      }
+      const int n_act = hi - lo;
+      const bool loads = fused || has_c;
+      const CUtensorMap* load_map = fused ? P.tma_p : P.tma_c;
+      const uint32_t load_bytes = fused ? 4096u : 2048u;
+      auto slot_of = [&](int q) { return (ring + (uint32_t)q) % nslot; };
+      auto issue_load = [&](int q) {   // lane 0: the operand sub-tile of active chunk q
+        const uint32_t sl = slot_of(q);
+        mbar_arrive_expect_tx(&cbar[sl], load_bytes);
+        tma_load_2d(stg + sl * slot_bytes, load_map, &cbar[sl], col0 + (lo + q) * 32, r0);
       };
-      auto next_active = [&](int c) {
-        int nx = c + 1;
-        while (nx < C::kTileN / 32 && !active(nx)) ++nx;
-        return nx < C::kTileN / 32 ? nx : -1;
-      };
-      const bool loads = ep.fused != 0 || has_c;
-      const uint32_t load_bytes = ep.fused ? 4096u : 2048u;
-      const CUtensorMap* load_map = ep.fused ? P.tma_p : P.tma_c;
-      auto issue_load = [&](int c, uint32_t st) {   // lane 0
-        mbar_arrive_expect_tx(&cbar[st], load_bytes);
-        tma_load_2d(stg + st * 4096u, load_map, &cbar[st], (int32_t)(tl.bj * C::kTileN + c * 32), r0);
-      };
+      if constexpr (CHAIN) {
+        // the addend (the Gram product) was written by other CTAs: the dependency the producer
+        // waited for also orders this warp's loads of it
+        const PhaseDesc& D = ca.phases[ph];
+        if (has_c && D.dep >= 0) {
+          if (lane == 0) {
+            counter_wait_bounded(ca.done + (size_t)D.dep * ca.nmats + P.mat, D.dep_target[P.mat], abort_flag, wait_ns);
+            fence_proxy_async_global();
+          }
+          __syncwarp();
+        }
+      }
+      if (loads && n_act > 0) {
+        // the stores of earlier tiles have read their slots; the first loads of this tile go out
+        if (lane == 0) {
+          bulk_wait_group_read<0>();
+          for (int q = 0; q < ahead && q < n_act; ++q) issue_load(q);
+        }
+        for (int q = 0; q < ahead && q < n_act; ++q) inflight |= 1u << slot_of(q);
+      }
       // TMEM loads run one 32-column chunk ahead of the arithmetic: the load of the next active
-      // chunk is issued before the current chunk is processed, and waited for after it. Chunks
-      // that produce no output (clipped, or below the diagonal of a symmetric output) are not
-      // loaded at all.
+      // chunk is issued before the current chunk is processed, and waited for after it.
       const uint32_t tmem_row = (quarter * 32u) << 16;
       auto tmem_col = [&](int c) { return (WIDE ? 0u : acc * 256u) + (uint32_t)c * 32u; };
       // one chunk whose accumulator values are in r; false when an operand-load wait gave up
@@ -394,55 +556,57 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[WIDE ? ch / 8 : acc]), 0));
         }
-        const int32_t c0 = (int32_t)(tl.bj * C::kTileN + ch * 32);
-        if (r0 >= (int32_t)P.M || c0 >= (int32_t)P.N) return true;        // fully clipped
-        if (P.sym && c0 + 32 <= r0) return true;                            // mirrored elsewhere
-        const bool diag_blk = P.sym && c0 == r0;
-        const bool mirror = P.sym && c0 >= r0 + 32;
-        uint8_t* direct = stg + set * 4096u;
-        uint8_t* mirr = direct + 2048u;
-        if (lane == 0) bulk_wait_group_read<1>();   // the store issued from this set has read it
-        __syncwarp();
+        if (ch < lo || ch >= hi) return true;
+        const int q = ch - lo;
+        const uint32_t sl = slot_of(q);
+        uint8_t* buf = stg + sl * slot_bytes;
+        const int32_t c0 = col0 + ch * 32;
+        const bool mirror = whole_sym && c0 >= r0 + 32;
+        uint8_t* mirr = buf + 2048u;   // the mirrored sub-tile's half of a 4 KB slot
         if (loads) {
-          const int nx = next_active(ch);
-          if (lane == 0) {
-            if (pend != ch) issue_load(ch, set);
-            if (nx >= 0) {
-              bulk_wait_group_read<0>();   // the other set's last store has read it too
-              issue_load(nx, set ^ 1u);
+          if (q + ahead < n_act) {
+            if (lane == 0) {
+              // that slot was last used by the store of active chunk q + ahead - nslot
+              if (g) bulk_wait_group_read<0>();
+              else bulk_wait_group_read<1>();
+              issue_load(q + ahead);
             }
+            inflight |= 1u << slot_of(q + ahead);
           }
-          inflight |= 1u << set;
-          if (nx >= 0) inflight |= 1u << (set ^ 1u);
-          pend = nx;
-          const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&cbar[set], (cph >> set) & 1u, abort_flag,
+          const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&cbar[sl], (cph >> sl) & 1u, abort_flag,
                                                                      wait_ns));
           if (!got) return false;
-          cph ^= 1u << set;
-          inflight &= ~(1u << set);
+          cph ^= 1u << sl;
+          inflight &= ~(1u << sl);
+        } else {
+          // this slot was last used by the store of active chunk q - nslot
+          if (lane == 0) {
+            if (g) bulk_wait_group_read<1>();
+            else bulk_wait_group_read<3>();
+          }
+          __syncwarp();
         }
-        if (ep.fused) {
-          // last update: the whole 4 KB set holds the 32 x 32 fp32 parameter sub-tile (128-byte
-          // swizzle); O stays in fp32 and is never stored
+        if (fused) {
+          // last update: the slot holds the 32 x 32 fp32 parameter sub-tile (128-byte swizzle); O
+          // stays in fp32 and is never stored
           const float step = ep.lr * P.rms * s1;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            float4* q = reinterpret_cast<float4*>(direct + (uint32_t)lane * 128u +
-                                                  ((((uint32_t)j) ^ ((uint32_t)lane & 7u)) << 4));
-            float4 pv = *q;
+            float4* qv = reinterpret_cast<float4*>(buf + (uint32_t)lane * 128u +
+                                                   ((((uint32_t)j) ^ ((uint32_t)lane & 7u)) << 4));
+            float4 pv = *qv;
             pv.x = pv.x * ep.decay - step * __uint_as_float(r[4 * j + 0]);
             pv.y = pv.y * ep.decay - step * __uint_as_float(r[4 * j + 1]);
             pv.z = pv.z * ep.decay - step * __uint_as_float(r[4 * j + 2]);
             pv.w = pv.w * ep.decay - step * __uint_as_float(r[4 * j + 3]);
-            *q = pv;
+            *qv = pv;
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(P.tma_p, direct, c0, r0);
+            tma_store_2d(P.tma_p, buf, c0, r0);
             bulk_commit_group();
           }
-          set ^= 1u;
           return true;
         }
         float v[32];
@@ -451,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (has_c) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint4 raw = *reinterpret_cast<const uint4*>(direct + sw64_chunk((uint32_t)lane, (uint32_t)j));
+            const uint4 raw = *reinterpret_cast<const uint4*>(buf + sw64_chunk((uint32_t)lane, (uint32_t)j));
             const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -460,9 +624,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               v[8 * j + 2 * i + 1] += ep.k_c * f.y;
             }
           }
-          __syncwarp();   // every lane has read its addend row before the buffer is overwritten
+          __syncwarp();   // every lane has read its addend row before the slot is overwritten
         }
-        if (diag_blk) {
+        if (P.sym && c0 == r0) {   // a diagonal sub-tile
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (i == lane) v[i] += ep.diag;
@@ -473,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
 #pragma unroll
           for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[8 * j + 2 * i], v[8 * j + 2 * i + 1]);
-          *reinterpret_cast<uint4*>(direct + sw64_chunk((uint32_t)lane, (uint32_t)j)) = raw;
+          *reinterpret_cast<uint4*>(buf + sw64_chunk((uint32_t)lane, (uint32_t)j)) = raw;
         }
         if (mirror) {
           // element (row lane, column i) goes to row i, column lane of the transposed box
@@ -486,23 +650,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(P.tma_d, direct, c0, r0);
+          tma_store_2d(P.tma_d, buf, c0, r0);
           if (mirror) tma_store_2d(P.tma_d, mirr, r0, c0);
           bulk_commit_group();
         }
-        set ^= 1u;
         return true;
       };
       auto step = [&](const uint32_t (&cur)[32], uint32_t (&nxt)[32], int ch) -> bool {
         __syncwarp();
-        if (ch + 1 < C::kTileN / 32 && active(ch + 1)) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(ch + 1), nxt);
+        if (ch + 1 >= lo && ch + 1 < hi) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(ch + 1), nxt);
         const bool ok = chunk(cur, ch);
         tmem_ld_wait();
         return ok;
       };
       uint32_t ra[32], rb[32];
       __syncwarp();
-      if (active(0)) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(0), ra);
+      if (lo == 0 && hi > 0) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(0), ra);
       tmem_ld_wait();
       bool chunks_ok = true;
 #pragma unroll 1
@@ -512,6 +675,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!chunks_ok) timed_out = true;
       if (timed_out) break;
+      ring = (ring + (uint32_t)n_act) % nslot;
+      if constexpr (CHAIN) {
+        // this warp's stores of the tile are complete: count them for the phases that read them
+        if (lane == 0) {
+          bulk_wait_group_all();
+          fence_proxy_async_global();
+          red_release_gpu_add(ca.done + (size_t)ph * ca.nmats + P.mat, 1u);
+        }
+        __syncwarp();
+      }
       if constexpr (WIDE) {
         acc_phase ^= 1u;
       } else if (++acc == 2) {
@@ -522,8 +695,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (timed_out && lane == 0) raise_abort(abort_flag, PAIR, rank);
     // loads still in flight (only after a timeout) must land before the CTA exits
     if (lane == 0)
-      for (uint32_t st = 0; st < 2; ++st)
-        if (inflight & (1u << st)) mbar_wait_bounded(&cbar[st], (cph >> st) & 1u, zero_flag, kTimeoutNs);
+      for (uint32_t sl = 0; sl < 4; ++sl)
+        if (inflight & (1u << sl)) mbar_wait_bounded(&cbar[sl], (cph >> sl) & 1u, zero_flag, kTimeoutNs);
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
   } else {
@@ -655,22 +828,23 @@ cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_
                            EpiScalars ep, int* status, int grid, cudaStream_t s) {
   using C = TcCfg<false>;
   static PerDeviceOnce once;
-  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<false, false>, (int)C::kSmemBytes, once);
+  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<false, false, false>, (int)C::kSmemBytes, once);
   if (e != cudaSuccess) return e;
   if (total_tiles == 0) return cudaSuccess;
   if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
-  ns_gemm_tc_kernel<false, false><<<grid, kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status);
+  ns_gemm_tc_kernel<false, false, false><<<grid, kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status,
+                                                                               ChainArgs{});
   return cudaGetLastError();
 }
 
 namespace {
 
-template <bool WIDE>
+template <bool WIDE, bool CHAIN>
 cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles, EpiScalars ep,
-                        int* status, int max_pairs, cudaStream_t s) {
+                        int* status, int max_pairs, cudaStream_t s, ChainArgs ca) {
   using C = TcCfg<true, WIDE>;
-  static PerDeviceOnce once;   // one per tile width
-  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<true, WIDE>, (int)C::kSmemBytes, once);
+  static PerDeviceOnce once;   // one per instantiation
+  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<true, WIDE, CHAIN>, (int)C::kSmemBytes, once);
   if (e != cudaSuccess) return e;
   if (total_tiles == 0) return cudaSuccess;
   const uint32_t pairs = (uint32_t)max_pairs < total_tiles ? (uint32_t)max_pairs : total_tiles;
@@ -686,26 +860,31 @@ cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_til
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ns_gemm_tc_kernel<true, WIDE>, probs, nprobs, total_tiles, ep, status);
+  return cudaLaunchKernelEx(&cfg, ns_gemm_tc_kernel<true, WIDE, CHAIN>, probs, nprobs, total_tiles, ep, status, ca);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                 EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
-  return launch_pair<false>(probs, nprobs, total_tiles, ep, status, max_pairs, s);
+  return launch_pair<false, false>(probs, nprobs, total_tiles, ep, status, max_pairs, s, ChainArgs{});
 }
 
 cudaError_t launch_gemm_tc_pair_wide(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                      EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
-  return launch_pair<true>(probs, nprobs, total_tiles, ep, status, max_pairs, s);
+  return launch_pair<true, false>(probs, nprobs, total_tiles, ep, status, max_pairs, s, ChainArgs{});
+}
+
+cudaError_t launch_gemm_tc_pair_chain(ChainArgs ca, uint32_t total_tiles, EpiScalars ep, int* status,
+                                      int max_pairs, cudaStream_t s) {
+  return launch_pair<false, true>(nullptr, 0, total_tiles, ep, status, max_pairs, s, ca);
 }
 
 // Largest number of CTA pairs of the paired kernel that can be resident at once.
 int gemm_tc_pair_capacity(int sms) {
   using C = TcCfg<true>;
   static_assert(TcCfg<true, true>::kSmemBytes == C::kSmemBytes, "both pair variants have one occupancy");
-  cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(ns_gemm_tc_kernel<true, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::kSmemBytes);
   if (e != cudaSuccess) return sms / 2;
   cudaLaunchConfig_t cfg = {};
@@ -720,7 +899,7 @@ int gemm_tc_pair_capacity(int sms) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  e = cudaOccupancyMaxActiveClusters(&n, ns_gemm_tc_kernel<true, false>, &cfg);
+  e = cudaOccupancyMaxActiveClusters(&n, ns_gemm_tc_kernel<true, false, false>, &cfg);
   if (e != cudaSuccess || n <= 0) {
     cudaGetLastError();
     return sms / 2;

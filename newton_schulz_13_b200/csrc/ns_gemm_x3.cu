@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, fills = 0;
       for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
         const Tile tl = decode_tile<kTileM, kTileN>(probs, nprobs, t);
-        const GemmProblemX3& P = probs[tl.p];
+        const GemmProblemX3 P = probs[tl.p];   // in registers: the asm below clobbers memory
         const uint32_t kblocks = (P.K + kX3BK - 1) / kX3BK;
         const int32_t a_row0 = (int32_t)(tl.bi * kTileM + rank * 128);
         const int32_t b_row0 = (int32_t)(tl.bj * kTileN + rank * 128);
@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       for (uint32_t t = unit; t < total_tiles && !timed_out; t += n_units) {
         const Tile tl = decode_tile<kTileM, kTileN>(probs, nprobs, t);
-        const GemmProblemX3& P = probs[tl.p];
+        const GemmProblemX3 P = probs[tl.p];   // in registers: the asm below clobbers memory
         const uint32_t kblocks = (P.K + kX3BK - 1) / kX3BK;
         const uint32_t idesc = idesc_tf32_f32(kTileM, kTileN, P.a_mn, P.b_mn);
         // 8 K per MMA: 32 bytes along a K-major row, or 8 rows of an MN-major box
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc = 0, acc_phase = 0;
     for (uint32_t t = unit; t < total_tiles; t += n_units) {
       const Tile tl = decode_tile<kTileM, kTileN>(probs, nprobs, t);
-      const GemmProblemX3& P = probs[tl.p];
+      const GemmProblemX3 P = probs[tl.p];   // in registers: the asm below clobbers memory
       const float alpha = (ep.e_acc | ep.e_c) ? *P.alpha : 1.0f;
       const float s_acc = ep.k_acc * alpha_pow(alpha, ep.e_acc);
       const float s_c = ep.k_c * alpha_pow(alpha, ep.e_c);
