@@ -235,15 +235,20 @@ MUON_API int muon_set_wave_elements(int64_t elements);
  * default.) Returns MUON_OK. */
 MUON_API int muon_set_wait_limit_ns(uint64_t ns);
 
-/* Tuning and diagnostics: nonzero (the default) runs the whole Newton-Schulz iteration of each
- * wave whose matrices all use 256 x 256 tiles (bf16 working precision; waves dominated by
- * matrices with min(rows, cols) >= 2048 use 256 x 512 tiles and are not affected) as one chained
- * launch: tiles are claimed in order, and each phase waits per matrix for the phase whose results
- * it reads, so the phases of different matrices overlap and small matrices are not launch-bound.
- * Zero launches one grouped kernel per phase. The results are bit-identical either way. With
- * chaining, muon_profile_read counts the whole iteration under MUON_KC_GEMM (no per-phase
- * breakdown). Returns MUON_OK. */
-MUON_API int muon_set_chained_launch(int on);
+/* Tuning and diagnostics: chained launches. A wave whose matrices all use 256 x 256 tiles (bf16
+ * working precision; waves dominated by matrices with min(rows, cols) >= 2048 use 256 x 512 tiles
+ * and are never chained) can run its whole Newton-Schulz iteration as one launch: tiles are
+ * claimed in order, and each phase waits per matrix for the phase whose results it reads, so the
+ * fixed cost of fifteen launches and their tails disappears.
+ *   mode 0: never chain; one grouped kernel per phase.
+ *   mode 1 (default): chain a wave when one iteration has at most 8 tiles per CTA pair of the
+ *           device (small sets of small matrices, where launch costs dominate).
+ *   mode 2: chain every wave of small matrices.
+ * The results are bit-identical in every mode. With chaining, muon_profile_read counts the whole
+ * iteration under MUON_KC_GEMM (no per-phase breakdown). Applies to calls made after it (a cached
+ * plan built in another mode is rebuilt). Returns MUON_OK, or MUON_ERR_INVALID_ARG for another
+ * mode. */
+MUON_API int muon_set_chained_launch(int mode);
 
 /* Kernel classes counted and timed by the library, indices into muon_profile_read's arrays. */
 enum {

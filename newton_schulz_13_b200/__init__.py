@@ -234,11 +234,11 @@ def set_wave_elements(elements: int = 0) -> None:
     _check(lib.muon_set_wave_elements(int(elements)))
 
 
-def set_chained_launch(on: bool = True) -> None:
-    """Whole Newton-Schulz iteration of a wave of small matrices as one chained launch (default),
-    or one launch per phase. Results are bit-identical; see muon_set_chained_launch in
-    include/muon.h."""
-    _check(lib.muon_set_chained_launch(int(on)))
+def set_chained_launch(mode: int = 1) -> None:
+    """Chained launches of a wave's whole Newton-Schulz iteration: 0 never, 1 (default) for waves
+    with at most 8 tiles per CTA pair per iteration, 2 for every wave of small matrices. Results
+    are bit-identical; see muon_set_chained_launch in include/muon.h."""
+    _check(lib.muon_set_chained_launch(int(mode)))
 
 
 def set_wait_limit_ns(ns: int = 0) -> None:

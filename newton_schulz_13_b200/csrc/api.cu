@@ -135,9 +135,14 @@ struct BufMapsX3 {   // TMA views of one two-plane fp32 buffer: K-major and MN-m
 constexpr int64_t kWaveElements = int64_t(1) << 29;
 int64_t g_wave_elements = kWaveElements;   // muon_set_wave_elements
 uint64_t g_wait_ns = 0;                     // muon_set_wait_limit_ns (0: the kernels' default)
-// Chained launches: a wave whose products all run on 256 x 256 bf16 tiles runs its whole
-// Newton-Schulz iteration (every phase of every step) as one launch (muon_set_chained_launch).
-bool g_chain = true;
+// Chained launches (muon_set_chained_launch): a wave whose products all run on 256 x 256 bf16
+// tiles may run its whole Newton-Schulz iteration (every phase of every step) as one launch.
+// Mode 0: never; 1 (default): when one iteration has at most kChainTilesPerPair tiles per CTA
+// pair, where the per-phase launches' fixed costs dominate (a single 256 x 512 matrix 0.31 ->
+// 0.18 ms, the cubic 12-matrix set 0.50 -> 0.38 ms), while waves with 25-30 tiles per pair per
+// iteration (GPT-2-small, Mamba) measured 2-4 % faster per phase; 2: always.
+int g_chain_mode = 1;
+constexpr uint32_t kChainTilesPerPair = 8;
 constexpr int kMaxChainPhases = 3 * MUON_MAX_NS_STEPS;
 
 // A wave: matrices [j0, j1) of the plan. Every prefix sum in the device tables (elementwise
@@ -146,6 +151,7 @@ constexpr int kMaxChainPhases = 3 * MUON_MAX_NS_STEPS;
 struct Wave {
   int j0 = 0, j1 = 0;
   bool wide = false;   // bf16 Gram and update products on 256 x 512 tiles (see build_plan)
+  bool chain = false;  // bf16: the iteration runs as one chained launch (g_chain_mode)
   int64_t n_chunks = 0, cs_items = 0, cm_items = 0;
   uint32_t tiles_gram = 0, tiles_poly = 0, tiles_upd = 0;
   double fl_gram = 0, fl_poly = 0, fl_upd = 0;      // nominal flops per launch
@@ -161,7 +167,7 @@ struct Plan {
   std::vector<Shape> shapes;
   int x_bf16 = 1;
   int64_t wave_elements = 0;
-  bool chain = false;        // built for chained launches (Gram problems in matrix order)
+  int chain_mode = 1;        // g_chain_mode the plan was built with
   uint64_t arena_gen = 0;
   char* tab = nullptr;       // this plan's tables (cudaMalloc)
   size_t tab_bytes = 0;
@@ -261,13 +267,13 @@ int device_state(DeviceState** out) {
 // round-robin over the CTA pairs in table order; a wave's Gram tiles differ in K (the longer side
 // of each matrix, up to 4x between the matrices of one model), so placing the longest tiles
 // first evens out the pairs' loads. Waves of large matrices (256 x 512 tiles, ten or more tiles
-// per pair) keep the matrix order, which measured faster there, and so do chained launches
-// (`chained`): they balance by claiming tiles as they go, and a Gram product in another order
-// than the update it waits for would start with the matrices whose updates finish last.
+// per pair) keep the matrix order, which measured faster there, and so do chained waves: they
+// balance by claiming tiles as they go, and a Gram product in another order than the update it
+// waits for would start with the matrices whose updates finish last.
 template <class Prob>
-void order_gram_by_k(std::vector<Prob>& probs, const std::vector<Wave>& waves, bool chained) {
+void order_gram_by_k(std::vector<Prob>& probs, const std::vector<Wave>& waves) {
   for (const Wave& w : waves) {
-    if (w.wide || chained) continue;
+    if (w.wide || w.chain) continue;
     std::stable_sort(probs.begin() + w.j0, probs.begin() + w.j1,
                      [](const Prob& a, const Prob& b) { return a.K > b.K; });
     uint32_t t = 0;
@@ -284,7 +290,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   for (size_t i = 0; i < ds.plans.size(); ++i) {
     const Plan& q = *ds.plans[i];
     if (q.shapes == shapes && q.x_bf16 == x_bf16 && q.wave_elements == g_wave_elements &&
-        q.chain == g_chain && q.arena_gen == ds.arena_gen) {
+        q.chain_mode == g_chain_mode && q.arena_gen == ds.arena_gen) {
       if (i > 0) std::rotate(ds.plans.begin(), ds.plans.begin() + i, ds.plans.begin() + i + 1);
       *out = ds.plans[0].get();
       return MUON_OK;
@@ -294,7 +300,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
   P->shapes = shapes;
   P->x_bf16 = x_bf16;
   P->wave_elements = g_wave_elements;
-  P->chain = g_chain;
+  P->chain_mode = g_chain_mode;
   const int n = (int)shapes.size();
   // bf16 mode: one bf16 plane per buffer; fp32 mode: hi and lo fp32 planes (GemmProblemX3)
   const size_t esz = x_bf16 ? 2 : 8;
@@ -585,8 +591,15 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       }
       MUON_CUDA(cudaMemcpy(P->d_tgt[0], tgt.data(), tgt.size() * 4, cudaMemcpyHostToDevice));
     }
-    order_gram_by_k(gram[0], P->waves, P->chain);
-    order_gram_by_k(gram[1], P->waves, P->chain);
+    // chained waves: small enough per iteration, and few enough matrices for the 16-bit index
+    for (Wave& w : P->waves) {
+      const uint32_t tiles = w.tiles_gram + w.tiles_poly + w.tiles_upd;
+      w.chain = !w.wide && n <= 65535 &&
+                (g_chain_mode == 2 ||
+                 (g_chain_mode == 1 && tiles <= kChainTilesPerPair * (uint32_t)std::max(1, ds.pair_capacity)));
+    }
+    order_gram_by_k(gram[0], P->waves);
+    order_gram_by_k(gram[1], P->waves);
     std::vector<GemmProblem>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
                       &P->d_updA[0], &P->d_updA[1]};
@@ -701,8 +714,8 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
     }
     if (bad) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(bad));
     MUON_CUDA(cudaMemcpy(d_maps, maps.data(), maps.size() * sizeof(CUtensorMap), cudaMemcpyHostToDevice));
-    order_gram_by_k(gram[0], P->waves, false);
-    order_gram_by_k(gram[1], P->waves, false);
+    order_gram_by_k(gram[0], P->waves);
+    order_gram_by_k(gram[1], P->waves);
     std::vector<GemmProblemX3>* lists[7] = {&gram[0], &gram[1], &poly, &updB[0], &updB[1], &updA[0], &updA[1]};
     void** dsts[7] = {&P->d_gram[0], &P->d_gram[1], &P->d_poly, &P->d_updB[0], &P->d_updB[1],
                       &P->d_updA[0], &P->d_updA[1]};
@@ -779,8 +792,11 @@ const void* fused_table(Plan& P, float* const* params, const std::vector<int>& i
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return nullptr;
-    probs[j].tma_p = P.d_pmaps + j;
-    probs[j].rms = rms[j];
+  }
+  for (int q = 0; q < n; ++q) {   // table position q holds the update of matrix probs[q].mat
+    const int j = probs[q].mat;
+    probs[q].tma_p = P.d_pmaps + j;
+    probs[q].rms = rms[j];
   }
   cudaError_t e = write_table(P.d_pmaps, maps.data(), n * sizeof(CUtensorMap), s, &g_launches);
   if (e == cudaSuccess) e = write_table(P.d_fused, probs.data(), n * sizeof(GemmProblem), s, &g_launches);
@@ -912,8 +928,7 @@ int run_ns_chained(DeviceState& ds, Plan& P, const Wave& w, int wave_idx, const 
 int run_ns(DeviceState& ds, Plan& P, const Wave& w, int wave_idx, const std::vector<muon_coeffs_t>& co,
            cudaStream_t s, const void* fused_last = nullptr, float lr = 0.0f, float decay = 1.0f) {
   const int n = w.j1 - w.j0;
-  if (P.x_bf16 && !w.wide && g_chain && !co.empty() && co.size() * 3 <= (size_t)kMaxChainPhases &&
-      P.shapes.size() <= 65535)
+  if (P.x_bf16 && w.chain && !co.empty() && co.size() * 3 <= (size_t)kMaxChainPhases)
     return run_ns_chained(ds, P, w, wave_idx, co, s, fused_last, lr, decay);
   // the wave's sub-range of a problem table
   auto tc = [&](void* t) { return static_cast<GemmProblem*>(t) + w.j0; };
@@ -1096,10 +1111,11 @@ int muon_set_wave_elements(int64_t elements) {
   return MUON_OK;
 }
 
-int muon_set_chained_launch(int on) {
+int muon_set_chained_launch(int mode) {
   std::lock_guard<std::mutex> lk(g_mu);
   t_err.clear();
-  g_chain = on != 0;
+  if (mode < 0 || mode > 2) return fail(MUON_ERR_INVALID_ARG, "mode must be 0, 1 or 2");
+  g_chain_mode = mode;
   return MUON_OK;
 }
 

@@ -5,10 +5,11 @@
 // One kernel template serves all three products. A launch is a list of independent problems (one
 // per matrix of a wave of the optimizer step, all at the same iteration and phase), each
 //     D = s_acc * (opA . opB^T) + s_c * C + diag I,
-// scheduled statically over a persistent grid. The Muon step uses the CTA-pair variants
-// (clusters of two CTAs on two SMs, tcgen05 cta_group::2): 256 x 256 tiles, or 256 x 512 "wide"
-// tiles for the Gram and update products of large matrices. A single-CTA variant (128 x 256
-// tiles) serves the no-allocation entry point. 192 threads per CTA:
+// scheduled statically over a persistent grid; or, chained, every phase of a wave's iteration in
+// one launch with tiles claimed in order (see CHAIN below). The Muon step uses the CTA-pair
+// variants (clusters of two CTAs on two SMs, tcgen05 cta_group::2): 256 x 256 tiles, or 256 x 512
+// "wide" tiles for the Gram and update products of large matrices. A single-CTA variant
+// (128 x 256 tiles) serves the no-allocation entry point. 192 threads per CTA:
 //   warp 0      TMA producer: 64-deep K slices of opA and opB into a shared-memory ring
 //               (128-byte swizzle), K-major or MN-major boxes per operand; in a pair each CTA
 //               loads its own 128 opA rows and its 128 of every 256 opB rows, and both CTAs'
@@ -20,9 +21,11 @@
 //   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, add s_c * C, round to bf16,
 //               stage 32 x 32 sub-tiles in shared memory and write them with TMA stores (pair),
 //               or store directly (single CTA). For the symmetric products (A = X X^T and
-//               A A = A A^T) only tiles that touch the upper triangle are computed, and the
-//               strictly-upper part is also written mirrored. The last update of a Muon step
-//               applies the parameter update instead of storing D.
+//               A A = A A^T) only tiles that touch the upper triangle are computed; the output
+//               is written whole (the strictly-upper part also mirrored) or, on waves of small
+//               matrices, in the upper-block form (only the 256-blocks on or above the diagonal;
+//               readers take K slices below the diagonal transposed). The last update of a Muon
+//               step applies the parameter update instead of storing D.
 // Both orientations of the iterate are read in place: a wide iterate X (m x n) is K-major for
 // X X^T and MN-major as the right operand of B X; a tall stored matrix G (n x m, iterate G^T)
 // is MN-major for G^T G and K-major for G B. So no transposed copies are ever made.
@@ -184,6 +187,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the tile index with a stride of n_units. Chained launches: the even CTA's producer (claimer)
   // takes the next index with an atomic add and queues it in both CTAs; the other roles read it
   // from their CTA's queue (warp_wide: every lane of an epilogue warp) and release the entry.
+  // The claimer reserves one tile ahead: the atomic for the following tile goes out when a tile
+  // is handed out, so its latency overlaps that tile's loads instead of stalling the producer.
+  uint32_t reserved = kNoTile;
+  bool have_reserved = false;
   auto next_tile = [&](uint32_t& seq, uint32_t& t, bool claimer, bool warp_wide) -> bool {
     if constexpr (!CHAIN) {
       t = unit + seq * n_units;
@@ -196,8 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           timed_out = true;
           return false;
         }
-        uint32_t v = atomicAdd(ca.tile_counter, 1u);
+        uint32_t v = have_reserved ? reserved : atomicAdd(ca.tile_counter, 1u);
         if (v >= total_tiles) v = kNoTile;
+        have_reserved = v != kNoTile;
+        if (have_reserved) reserved = atomicAdd(ca.tile_counter, 1u);   // used at the next call
         tq[q] = v;
         st_shared_cluster(mapa_shared(smem_u32((const void*)&tq[q]), 1u), v);
         mbar_arrive(&tq_full[q]);
@@ -247,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int issued_parity[C::kStages];
       for (int s = 0; s < C::kStages; ++s) issued_parity[s] = -1;
       uint32_t stage = 0, phase = 0, fills = 0, seq = 0, t = 0;
+      uint32_t dep_done = 0xffffffffu;   // chained: last (phase, matrix) dependency seen complete
       while (!timed_out && next_tile(seq, t, leader, false)) {
         Tile tl;
         const GemmProblem* Pp;
@@ -259,13 +269,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (CHAIN) {
           // the results this tile reads (same matrix, earlier phase) must be complete
           const PhaseDesc& D = ca.phases[ph];
-          if (D.dep >= 0) {
+          // completion counts only grow: a dependency seen complete stays complete
+          const uint32_t key = ((uint32_t)D.dep << 16) | P.mat;
+          if (D.dep >= 0 && key != dep_done) {
             if (!counter_wait_bounded(ca.done + (size_t)D.dep * ca.nmats + P.mat, D.dep_target[P.mat], abort_flag,
                                       wait_ns)) {
               timed_out = true;
               break;
             }
             fence_proxy_async_global();
+            dep_done = key;
           }
         }
         const uint32_t kblocks = (P.K + kTcBK - 1) / kTcBK;
@@ -472,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t ring = 0;       // slot of the next active chunk
     int geo = -1;            // slot geometry in use: 0 four 2 KB slots, 1 two 4 KB slots
     uint32_t acc = 0, acc_phase = 0, seq = 0, t = 0;
+    uint32_t dep_done = 0xffffffffu;   // chained: last (phase, matrix) dependency seen complete
     while (next_tile(seq, t, false, true)) {
       Tile tl;
       const GemmProblem* Pp;
@@ -527,12 +541,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the addend (the Gram product) was written by other CTAs: the dependency the producer
         // waited for also orders this warp's loads of it
         const PhaseDesc& D = ca.phases[ph];
-        if (has_c && D.dep >= 0) {
+        const uint32_t key = ((uint32_t)D.dep << 16) | P.mat;
+        if (has_c && D.dep >= 0 && key != dep_done) {
           if (lane == 0) {
             counter_wait_bounded(ca.done + (size_t)D.dep * ca.nmats + P.mat, D.dep_target[P.mat], abort_flag, wait_ns);
             fence_proxy_async_global();
           }
           __syncwarp();
+          dep_done = key;
         }
       }
       if (loads && n_act > 0) {
@@ -678,6 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ring = (ring + (uint32_t)n_act) % nslot;
       if constexpr (CHAIN) {
         // this warp's stores of the tile are complete: count them for the phases that read them
+        // (publishing at once measured faster than collecting several tiles per publication)
         if (lane == 0) {
           bulk_wait_group_all();
           fence_proxy_async_global();

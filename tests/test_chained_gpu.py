@@ -4,8 +4,9 @@ tiles claimed in order and each phase waiting per matrix for the phase whose res
 The chained launch runs the same tiles with the same arithmetic as one launch per phase, so the
 results must be bit-identical; every workload whose waves use 256 x 256 tiles is checked both
 ways over two steps (the quintic, cubic with zero-centring, where the update waits on the Gram
-product directly, and the 8 + 2 hybrid schedule), and against the fp64 oracle through the
-workload tests, which run chained by default.
+product directly, and the 8 + 2 hybrid schedule). The automatic mode's choice per workload is
+checked by counting product launches; the workload tests check both paths against the fp64
+oracle (single_256x512 and the cubic set chain by default, the others do not).
 """
 import pytest
 import torch
@@ -20,12 +21,12 @@ pytestmark = pytest.mark.gpu
 def chain_switch():
     import newton_schulz_13_b200 as ns
     yield ns.set_chained_launch
-    ns.set_chained_launch(True)
+    ns.set_chained_launch(1)
 
 
-def _run(wl, chained, coeffs=None, prec="bf16"):
+def _run(wl, mode, coeffs=None, prec="bf16"):
     import newton_schulz_13_b200 as ns
-    ns.set_chained_launch(chained)
+    ns.set_chained_launch(mode)
     case = StepCase(wl, sample=[], device_fill=True)
     for k in range(2):
         case.step(k, prec=prec, coeffs=coeffs)
@@ -39,16 +40,14 @@ def _run(wl, chained, coeffs=None, prec="bf16"):
 def test_chained_launch_is_bit_identical_to_per_phase_launches(chain_switch, name, sched):
     wl = synth.WORKLOADS[name]
     coeffs = synth.HYBRID if sched == "hybrid" else None
-    a = _run(wl, True, coeffs)
-    b = _run(wl, False, coeffs)
+    a = _run(wl, 2, coeffs)   # chained
+    b = _run(wl, 0, coeffs)   # one launch per phase
     for x, y in zip(a, b):
         assert torch.equal(x, y)
 
 
-def test_chained_launch_counts_one_product_launch_per_wave(chain_switch):
-    """GPT-2-small is one wave: one chained launch replaces the fifteen per-phase launches."""
+def _product_launches(wl):
     import newton_schulz_13_b200 as ns
-    wl = synth.WORKLOADS["gpt2_small"]
     case = StepCase(wl, sample=[], device_fill=True)
     case.step(0)                      # builds the plan and writes the tables
     torch.cuda.synchronize()
@@ -60,5 +59,23 @@ def test_chained_launch_counts_one_product_launch_per_wave(chain_switch):
         rec = ns.profile_read()
     finally:
         ns.profile_enable(False)
-    assert rec["gemm"][0] == 1, rec["gemm"]
     assert ns.check_status() == ns.OK
+    return rec["gemm"][0]
+
+
+@pytest.mark.parametrize("name,mode,launches", [
+    ("gpt2_small", 2, 1),        # forced: one chained launch replaces the fifteen per-phase ones
+    ("gpt2_small", 1, 15),       # automatic: about 25 tiles per CTA pair per iteration, per phase
+    ("gpt2_small", 0, 15),
+    ("single_256x512", 1, 1),    # automatic: a handful of tiles, chained
+    ("cubic_zero_center_12", 1, 1),
+    ("cubic_zero_center_12", 0, 10)])   # cubic: no polynomial product, two launches per step
+def test_chained_launch_choice(chain_switch, name, mode, launches):
+    chain_switch(mode)
+    assert _product_launches(synth.WORKLOADS[name]) == launches
+
+
+def test_chain_mode_rejects_other_values():
+    import newton_schulz_13_b200 as ns
+    with pytest.raises(ns.MuonError):
+        ns.set_chained_launch(3)
