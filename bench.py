@@ -235,7 +235,7 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     ns.set_wave_elements(args.wave_elements)
-    ns.set_chained_launch(1 if args.chain else 0)
+    ns.set_chained_launch(args.chained_launch)
     if world > 1:
         import torch.distributed as dist
         import datetime
@@ -349,8 +349,8 @@ def run_ours(args, world, rank, local):
                          "126 MB L2" % (elements * (4 + 4 + 2 * gbytes) / 1e9),
                    "muon_step_calls_per_step": len(call_groups),
                    "wave_elements": args.wave_elements or (1 << 29),
-                   "chained_launch": "auto (waves with <= 8 tiles per CTA pair per iteration)"
-                                     if args.chain else "off",
+                   "chained_launch": ("off", "auto (waves with <= 8 tiles per CTA pair per iteration)",
+                                      "every wave")[args.chained_launch],
                    "parallelism": ("one weight set split across GPUs by Newton-Schulz FLOPs, updated parameters "
                                    "all-gathered (strong scaling)") if args.sharded else
                                   "independent weight set per GPU (weak scaling, no collective)"},
@@ -611,9 +611,9 @@ def main(argv=None):
     ap.add_argument("--step-group-layers", type=int, default=0,
                     help="device-timed step as one muon_step call per group of this many layers "
                          "(0: one call over all matrices)")
-    ap.add_argument("--no-chain", dest="chain", action="store_false",
-                    help="one launch per Newton-Schulz phase for every wave, instead of the default "
-                         "chained launch of small waves (see muon_set_chained_launch)")
+    ap.add_argument("--chained-launch", type=int, choices=(0, 1, 2), default=1,
+                    help="0: one launch per Newton-Schulz phase; 1 (default): the whole iteration of a "
+                         "small wave in one launch; 2: every wave chained (see muon_set_chained_launch)")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-group-layers", type=int, default=1,
