@@ -517,7 +517,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
         g.tiles_m = (uint32_t)ceil_div(m, kTcPairBM);
         g.tiles_n = (uint32_t)ceil_div(m, w.wide ? kTcWideBN : kTcBN);
         g.sym = w.wide ? 1 : 2;   // A whole (mirrored writes) or in the upper-block form
-        g.mat = (uint16_t)j;
+        g.mat = (uint32_t)j;
         g.n_tiles = (uint32_t)(w.wide ? sym_tiles_wide(m) : sym_tiles(m));
         g.tile_begin = tg;
         gram[p].push_back(g);
@@ -526,7 +526,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
           GemmProblem u{};
           // B (or A) in the upper-block form: K slices below its diagonal blocks are read
           // transposed through its MN-major view
-          const uint8_t half = w.wide ? 0 : 1;
+          const uint32_t half = w.wide ? 0 : 1;
           if (!tall) {
             u.tma_a = M_(mS.k128); u.a_mn = 0;
             u.tma_a_t = M_(mS.mn64); u.a_half = half;
@@ -541,7 +541,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
           u.tma_d = M_(mx[1 - p].st32);
           u.alpha = P->alpha[j];
           u.M = (uint32_t)r; u.N = (uint32_t)c; u.K = (uint32_t)m;
-          u.mat = (uint16_t)j;
+          u.mat = (uint32_t)j;
           u.tiles_m = (uint32_t)ceil_div(r, kTcPairBM);
           u.tiles_n = (uint32_t)ceil_div(c, w.wide ? kTcWideBN : kTcBN);
           u.n_tiles = u.tiles_m * u.tiles_n;
@@ -555,7 +555,7 @@ int build_plan(DeviceState& ds, const std::vector<Shape>& shapes, int x_bf16, Pl
       q.tma_a = M_(mA.k128); q.tma_b = M_(mA.k128);
       q.tma_a_t = M_(mA.mn64); q.tma_b_t = M_(mA.mn64);
       q.a_half = q.b_half = w.wide ? 0 : 1;
-      q.mat = (uint16_t)j;
+      q.mat = (uint32_t)j;
       q.d = static_cast<__nv_bfloat16*>(P->B[j]); q.ldd = P->ldm[j];
       q.tma_d = M_(mB.st32);
       q.tma_c = M_(mA.st32);

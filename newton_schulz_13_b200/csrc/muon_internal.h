@@ -81,16 +81,17 @@ struct GemmProblem {
   uint32_t tile_begin;      // prefix sum over the problems of the launch
   uint32_t n_tiles;
   float rms;                // fused last update: RMS factor s of this matrix
-  uint8_t a_mn, b_mn;       // 1: operand is MN-major
-  uint8_t sym;              // D is symmetric: compute the tiles touching the upper triangle, and
+  // The flags are full 32-bit words: with byte-sized fields, one kernel build read a_half out of
+  // the tile record's register copy wrongly (it saw b_mn there) in its MMA-issuing thread.
+  uint32_t a_mn, b_mn;      // 1: operand is MN-major
+  uint32_t sym;             // D is symmetric: compute the tiles touching the upper triangle, and
                             //   1: write the strictly-upper part also mirrored (whole matrix);
                             //   2 (CTA-pair kernel): write only the 256 x 256 blocks on or above
                             //      the diagonal (the upper-block form)
-  uint8_t a_half, b_half;   // 1 (CTA-pair kernel): the operand is a symmetric matrix in the
+  uint32_t a_half, b_half;  // 1 (CTA-pair kernel): the operand is a symmetric matrix in the
                             //   upper-block form; a K slice in a 256-block below the operand rows'
                             //   block is read transposed, from the mirror block, through tma_*_t
-  uint8_t pad;
-  uint16_t mat;             // chained launch: the problem's matrix (index within its plan)
+  uint32_t mat;             // chained launch: the problem's matrix (index within its plan)
 };
 
 // fp32 precision mode ("3xTF32"). Every fp32 matrix of the iteration is held as two planes of
@@ -114,9 +115,9 @@ struct GemmProblemX3 {
   uint32_t tile_begin;
   uint32_t n_tiles;
   float rms;                // fused last update: RMS factor s of this matrix
-  uint8_t a_mn, b_mn;       // 1: operand is MN-major
-  uint8_t sym;              // 1: D is symmetric (upper-triangle tiles, strictly-upper part mirrored)
-  uint8_t p_vec;            // 1: p rows are 16-byte aligned (ldp % 4 == 0, p 16-byte aligned)
+  uint32_t a_mn, b_mn;      // 1: operand is MN-major (32-bit words, as in GemmProblem)
+  uint32_t sym;             // 1: D is symmetric (upper-triangle tiles, strictly-upper part mirrored)
+  uint32_t p_vec;           // 1: p rows are 16-byte aligned (ldp % 4 == 0, p 16-byte aligned)
 };
 
 // Epilogue scalars of one launch: D = k_acc alpha^e_acc acc + k_c alpha^e_c C + diag I

@@ -9,7 +9,8 @@
 // one launch with tiles claimed in order (see CHAIN below). The Muon step uses the CTA-pair
 // variants (clusters of two CTAs on two SMs, tcgen05 cta_group::2): 256 x 256 tiles, or 256 x 512
 // "wide" tiles for the Gram and update products of large matrices. A single-CTA variant
-// (128 x 256 tiles) serves the no-allocation entry point. 192 threads per CTA:
+// (128 x 256 tiles) serves the no-allocation entry point. 192 threads per CTA (320 for the wide
+// tile, whose epilogue has eight warps):
 //   warp 0      TMA producer: 64-deep K slices of opA and opB into a shared-memory ring
 //               (128-byte swizzle), K-major or MN-major boxes per operand; in a pair each CTA
 //               loads its own 128 opA rows and its 128 of every 256 opB rows, and both CTAs'
@@ -18,7 +19,7 @@
 //               accumulation in tensor memory; 256 x 256 tiles alternate between two
 //               accumulators, so the epilogue of one tile overlaps the MMAs of the next, and
 //               wide tiles use both 256-column slots as the two halves of one accumulator;
-//   warps 2-5   epilogue: tcgen05.ld of the accumulator, scale, add s_c * C, round to bf16,
+//   warps 2-5   epilogue (2-9 for the wide tile): tcgen05.ld of the accumulator, scale, add s_c * C, round to bf16,
 //               stage 32 x 32 sub-tiles in shared memory and write them with TMA stores (pair),
 //               or store directly (single CTA). For the symmetric products (A = X X^T and
 //               A A = A A^T) only tiles that touch the upper triangle are computed; the output
@@ -50,7 +51,6 @@ namespace muon {
 namespace {
 
 constexpr uint32_t kBoxBytes = 64 * 64 * 2;  // one MN-major box: 64 K rows x 64 M/N columns
-constexpr int kThreads = 192;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // Geometry of the variants. Each CTA owns 128 accumulator rows; tensor memory holds 512 columns.
@@ -62,8 +62,10 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 //   CTA pair, wide: output tile 256 x 512 as two 256-column halves; each CTA loads its 128 rows of
 //                opA and 128 opB rows per half, and every opA slice feeds two MMAs (one per half):
 //                a quarter fewer operand bytes per FLOP than the 256 x 256 tile. The halves are
-//                the two 256-column slots of tensor memory (one accumulator); the epilogue drains
-//                half 0 first, so the next tile's half-0 MMAs overlap the drain of half 1.
+//                the two 256-column slots of tensor memory (one accumulator), so the next tile's
+//                MMAs wait for the drain: eight epilogue warps (two per 32-lane quarter of tensor
+//                memory, each taking alternate groups of four 32-column chunks) drain half 0
+//                first, and the next tile's half-0 MMAs overlap the drain of half 1.
 template <bool PAIR, bool WIDE = false>
 struct TcCfg {
   static_assert(PAIR || !WIDE, "the wide tile is a CTA-pair tile");
@@ -77,14 +79,23 @@ struct TcCfg {
   static constexpr uint32_t kBBytes = kBRows * kTcBK * 2;
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kEpiArrivals = PAIR ? 8 : 4;
-  // CTA pair: 8 KB of staging per epilogue warp (four 32 x 32 bf16 sub-tiles, or two fp32 ones)
-  static constexpr uint32_t kStagingPerWarp = 4 * 2048;
-  static constexpr uint32_t kStagingBytes = PAIR ? 4 * kStagingPerWarp : 0;
+  // warps: TMA producer, MMA issuer, then the epilogue warps
+  static constexpr int kEpiWarps = WIDE ? 8 : 4;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kWarpChunks = 8;   // 32-column chunks per epilogue warp and tile
+  static_assert(kWarpChunks * 32 * (kEpiWarps / 4) == kTileN, "chunks per warp");
+  // arrivals that free a 256-column accumulator slot: every epilogue warp of both CTAs
+  static constexpr uint32_t kEpiArrivals = PAIR ? 2 * kEpiWarps : kEpiWarps;
+  // CTA pair: staging per epilogue warp in 2 KB slots (a 32 x 32 bf16 sub-tile each; two make a
+  // slot for an fp32 sub-tile or a sub-tile and its mirror), 32 KB in all
+  static constexpr uint32_t kSlots = WIDE ? 2 : 4;
+  static constexpr uint32_t kStagingPerWarp = kSlots * 2048;
+  static constexpr uint32_t kStagingBytes = PAIR ? kEpiWarps * kStagingPerWarp : 0;
   static constexpr size_t kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 512;
   // the 512-byte tail: full and empty per stage, tfull and tempty per accumulator, drain, 16
-  // epilogue operand-load barriers (4 per epilogue warp) and the tile queue's 2 x 8 barriers; then
-  // the tensor-memory address, two flags, the producer's fill count and the 8 queued tiles
+  // epilogue operand-load barriers (one per staging slot) and the tile queue's 2 x 8 barriers;
+  // then the tensor-memory address, two flags, the producer's fill count and the 8 queued tiles
+  static_assert(kEpiWarps * kSlots == 16, "operand-load barriers");
   static_assert((2 * kStages + 2 + 2 + 33) * 8 + 12 * 4 <= 512, "barrier area");
   static_assert(kSmemBytes <= 232448, "dynamic shared memory per CTA");
 };
@@ -93,7 +104,7 @@ struct TcCfg {
 // symmetric operand in the upper-block form (half), when the slice's 256-block of K lies below the
 // 256-block `rblk` of the operand's rows, where only the mirror block (K rows, operand columns) is
 // stored. Both CTAs of a pair and every 16-deep MMA of a slice make the same choice.
-__device__ __forceinline__ bool slice_mn(uint8_t mn, uint8_t half, uint32_t kb, uint32_t rblk) {
+__device__ __forceinline__ bool slice_mn(uint32_t mn, uint32_t half, uint32_t kb, uint32_t rblk) {
   return mn || (half && (kb * (uint32_t)kTcBK) / 256u < rblk);
 }
 
@@ -116,7 +127,7 @@ constexpr uint32_t kNoTile = 0xffffffffu;
 // claimed tile depends only on tiles claimed before it, so the launch makes progress whether or
 // not all of its CTAs are resident.
 template <bool PAIR, bool WIDE, bool CHAIN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(TcCfg<PAIR, WIDE>::kThreads, 1)
     ns_gemm_tc_kernel(const GemmProblem* __restrict__ probs, int nprobs, uint32_t total_tiles,
                       EpiScalars ep, int* __restrict__ status, ChainArgs ca) {
   static_assert(!CHAIN || (PAIR && !WIDE), "chained launches use 256 x 256 CTA-pair tiles");
@@ -471,19 +482,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     // staged transposed and stored at the mirrored position, those strictly below are skipped)
     // or in the upper-block form (sym 2: chunks in a 256-block below the diagonal are skipped).
     // The chunks a tile writes ("active") are one contiguous range.
-    // Staging is a ring of slots per warp (8 KB) that the active chunks use in turn: four 2 KB
-    // slots (bf16 sub-tiles), or two 4 KB slots for the fused last update (fp32 parameter
-    // sub-tiles) and for whole symmetric outputs (a sub-tile and its mirror). A chunk that reads an
-    // operand sub-tile (the addend C, or the parameters) has its load issued `ahead` active chunks
-    // earlier (2 with 2 KB slots, 1 with 4 KB slots) into the slot it will use, once the store
-    // that used that slot last has read it.
+    // A warp takes 8 of the tile's 32-column chunks: all of them (256-column tile), or (wide
+    // tile, two warps per quarter) alternate groups of four, so that half 0 is drained first by
+    // both. The warp's active chunks are one contiguous run of its own list.
+    // Staging is a ring of 2 KB slots per warp (four; two for the wide tile's eight warps) that the
+    // active chunks use in turn: one slot per bf16 sub-tile, or pairs of slots for the fused last
+    // update (fp32 parameter sub-tiles) and for whole symmetric outputs (a sub-tile and its
+    // mirror). A chunk that reads an operand sub-tile (the addend C, or the parameters) has its
+    // load issued `ahead` active chunks earlier into the slot it will use (half the ring with 2 KB
+    // slots, one less than the ring with 4 KB slots), once the store that used that slot last has
+    // read it.
     const uint32_t quarter = (uint32_t)(warp & 3);
+    const uint32_t sub = (uint32_t)(warp - 2) >> 2;   // wide tile: which groups of four chunks
+    auto ch_of = [&](int i) -> int { return WIDE ? ((i >> 2) << 3) + (int)(sub << 2) + (i & 3) : i; };
     uint8_t* stg = staging + (uint32_t)(warp - 2) * C::kStagingPerWarp;
-    uint64_t* cbar = drain + 1 + 4 * (warp - 2);   // this warp's operand-load barriers, one per slot
+    uint64_t* cbar = drain + 1 + C::kSlots * (warp - 2);   // this warp's operand-load barriers, one per slot
     uint32_t cph = 0;        // bit s: phase of cbar[s]
     uint32_t inflight = 0;   // bit s: a load into slot s not yet waited for
     uint32_t ring = 0;       // slot of the next active chunk
-    int geo = -1;            // slot geometry in use: 0 four 2 KB slots, 1 two 4 KB slots
+    int geo = -1;            // slot geometry in use: 0 2 KB slots, 1 4 KB slots
     uint32_t acc = 0, acc_phase = 0, seq = 0, t = 0;
     uint32_t dep_done = 0xffffffffu;   // chained: last (phase, matrix) dependency seen complete
     while (next_tile(seq, t, false, true)) {
@@ -516,8 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ring = 0;
         geo = g;
       }
-      const uint32_t nslot = g ? 2u : 4u, slot_bytes = g ? 4096u : 2048u;
-      const int ahead = g ? 1 : 2;
+      const uint32_t nslot = g ? C::kSlots / 2 : C::kSlots, slot_bytes = g ? 4096u : 2048u;
+      const int ahead = g ? (int)nslot - 1 : (int)nslot / 2;
       // active chunks [lo, hi): inside the matrix and, for a symmetric output, not below the
       // 32 x 32 diagonal (whole form) or in a 256-block on or above the diagonal (upper-block
       // form); the same for every lane
@@ -527,7 +544,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int32_t first = whole_sym ? r0 : (P.sym ? (int32_t)(tl.bi * C::kTileM) : col0);
         lo = min(hi, max(0, (first - col0) / 32));
       }
-      const int n_act = hi - lo;
+      // this warp's active chunks: positions [i_lo, i_hi) of its list
+      int i_lo = 0, i_hi = 0;
+#pragma unroll
+      for (int i = 0; i < C::kWarpChunks; ++i) {
+        i_lo += ch_of(i) < lo ? 1 : 0;
+        i_hi += ch_of(i) < hi ? 1 : 0;
+      }
+      const int n_act = i_hi - i_lo;
       const bool loads = fused || has_c;
       const CUtensorMap* load_map = fused ? P.tma_p : P.tma_c;
       const uint32_t load_bytes = fused ? 4096u : 2048u;
@@ -535,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_load = [&](int q) {   // lane 0: the operand sub-tile of active chunk q
         const uint32_t sl = slot_of(q);
         mbar_arrive_expect_tx(&cbar[sl], load_bytes);
-        tma_load_2d(stg + sl * slot_bytes, load_map, &cbar[sl], col0 + (lo + q) * 32, r0);
+        tma_load_2d(stg + sl * slot_bytes, load_map, &cbar[sl], col0 + ch_of(i_lo + q) * 32, r0);
       };
       if constexpr (CHAIN) {
         // the addend (the Gram product) was written by other CTAs: the dependency the producer
@@ -559,21 +583,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int q = 0; q < ahead && q < n_act; ++q) inflight |= 1u << slot_of(q);
       }
-      // TMEM loads run one 32-column chunk ahead of the arithmetic: the load of the next active
-      // chunk is issued before the current chunk is processed, and waited for after it.
       const uint32_t tmem_row = (quarter * 32u) << 16;
       auto tmem_col = [&](int c) { return (WIDE ? 0u : acc * 256u) + (uint32_t)c * 32u; };
-      // one chunk whose accumulator values are in r; false when an operand-load wait gave up
-      auto chunk = [&](const uint32_t (&r)[32], int ch) -> bool {
-        // a 256-column slot is free once its last chunk is in registers (wide: half 0 after
-        // chunk 7, so the next tile's half-0 MMAs can start while half 1 drains)
-        if (ch % 8 == 7) {
+      // chunk i of this warp's list, whose accumulator values are in r; false when an operand-load
+      // wait gave up
+      auto chunk = [&](const uint32_t (&r)[32], int i) -> bool {
+        // a 256-column slot is free once its last chunks are in registers (wide: half 0 after
+        // each warp's first four, so the next tile's half-0 MMAs can start while half 1 drains)
+        if (WIDE ? (i & 3) == 3 : i == C::kWarpChunks - 1) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[WIDE ? ch / 8 : acc]), 0));
+          if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[WIDE ? i >> 2 : acc]), 0));
         }
-        if (ch < lo || ch >= hi) return true;
-        const int q = ch - lo;
+        if (i < i_lo || i >= i_hi) return true;
+        const int q = i - i_lo;
+        const int ch = ch_of(i);
         const uint32_t sl = slot_of(q);
         uint8_t* buf = stg + sl * slot_bytes;
         const int32_t c0 = col0 + ch * 32;
@@ -583,8 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (q + ahead < n_act) {
             if (lane == 0) {
               // that slot was last used by the store of active chunk q + ahead - nslot
-              if (g) bulk_wait_group_read<0>();
-              else bulk_wait_group_read<1>();
+              bulk_wait_group_read_upto(nslot - ahead - 1);
               issue_load(q + ahead);
             }
             inflight |= 1u << slot_of(q + ahead);
@@ -596,10 +619,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           inflight &= ~(1u << sl);
         } else {
           // this slot was last used by the store of active chunk q - nslot
-          if (lane == 0) {
-            if (g) bulk_wait_group_read<1>();
-            else bulk_wait_group_read<3>();
-          }
+          if (lane == 0) bulk_wait_group_read_upto(nslot - 1);
           __syncwarp();
         }
         if (fused) {
@@ -672,22 +692,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return true;
       };
-      auto step = [&](const uint32_t (&cur)[32], uint32_t (&nxt)[32], int ch) -> bool {
-        __syncwarp();
-        if (ch + 1 >= lo && ch + 1 < hi) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(ch + 1), nxt);
-        const bool ok = chunk(cur, ch);
-        tmem_ld_wait();
-        return ok;
-      };
-      uint32_t ra[32], rb[32];
-      __syncwarp();
-      if (lo == 0 && hi > 0) tmem_ld_32x32b_x32(tmem_base + tmem_row + tmem_col(0), ra);
-      tmem_ld_wait();
       bool chunks_ok = true;
 #pragma unroll 1
-      for (int ch = 0; ch < C::kTileN / 32 && chunks_ok; ch += 2) {   // kTileN / 32 is even
-        chunks_ok = step(ra, rb, ch);
-        if (chunks_ok) chunks_ok = step(rb, ra, ch + 1);
+      for (int i = 0; i < C::kWarpChunks && chunks_ok; ++i) {
+        uint32_t r[32];
+        __syncwarp();
+        if (i >= i_lo && i < i_hi) tmem_ld_32x32b_x32_sync(tmem_base + tmem_row + tmem_col(ch_of(i)), r);
+        chunks_ok = chunk(r, i);
       }
       if (!chunks_ok) timed_out = true;
       if (timed_out) break;
@@ -712,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (timed_out && lane == 0) raise_abort(abort_flag, PAIR, rank);
     // loads still in flight (only after a timeout) must land before the CTA exits
     if (lane == 0)
-      for (uint32_t sl = 0; sl < 4; ++sl)
+      for (uint32_t sl = 0; sl < C::kSlots; ++sl)
         if (inflight & (1u << sl)) mbar_wait_bounded(&cbar[sl], (cph >> sl) & 1u, zero_flag, kTimeoutNs);
     if (lane == 0) bulk_wait_group_all();
     __syncwarp();
@@ -743,8 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ch = 0; ch < C::kTileN / 32; ++ch) {
         uint32_t r[32];
         __syncwarp();
-        tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + acc * C::kTileN + ch * 32, r);
-        tmem_ld_wait();
+        tmem_ld_32x32b_x32_sync(tmem_base + ((quarter * 32u) << 16) + acc * C::kTileN + ch * 32, r);
         if (ch == C::kTileN / 32 - 1) {
           tc_fence_before();
           __syncwarp();
@@ -849,7 +859,7 @@ cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_
   if (e != cudaSuccess) return e;
   if (total_tiles == 0) return cudaSuccess;
   if ((uint32_t)grid > total_tiles) grid = (int)total_tiles;
-  ns_gemm_tc_kernel<false, false, false><<<grid, kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status,
+  ns_gemm_tc_kernel<false, false, false><<<grid, C::kThreads, C::kSmemBytes, s>>>(probs, nprobs, total_tiles, ep, status,
                                                                                ChainArgs{});
   return cudaGetLastError();
 }
@@ -867,7 +877,7 @@ cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_til
   const uint32_t pairs = (uint32_t)max_pairs < total_tiles ? (uint32_t)max_pairs : total_tiles;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -906,7 +916,7 @@ int gemm_tc_pair_capacity(int sms) {
   if (e != cudaSuccess) return sms / 2;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -267,8 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ch = 0; ch < kTileN / 32; ++ch) {
           uint32_t r[32];
           __syncwarp();
-          tmem_ld_32x32b_x32(tmem_base + ((quarter * 32u) << 16) + acc * kTileN + ch * 32, r);
-          tmem_ld_wait();
+          tmem_ld_32x32b_x32_sync(tmem_base + ((quarter * 32u) << 16) + acc * kTileN + ch * 32, r);
           if (ch == kTileN / 32 - 1) {
             tc_fence_before();
             __syncwarp();

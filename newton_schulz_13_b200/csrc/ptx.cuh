@@ -224,6 +224,14 @@ __device__ __forceinline__ void bulk_wait_group_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
 }
 
+// bulk_wait_group_read with a run-time bound n (0 to 3; larger values wait as for 3).
+__device__ __forceinline__ void bulk_wait_group_read_upto(uint32_t n) {
+  if (n == 0) bulk_wait_group_read<0>();
+  else if (n == 1) bulk_wait_group_read<1>();
+  else if (n == 2) bulk_wait_group_read<2>();
+  else bulk_wait_group_read<3>();
+}
+
 // Waits until all of this thread's committed bulk groups have completed.
 __device__ __forceinline__ void bulk_wait_group_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -273,22 +281,23 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
       : "memory");
 }
 
-// 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (base lane + t).
-__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+// 32 lanes x 32 consecutive 32-bit columns: thread t of the warp gets lane (base lane + t). The
+// load and its wait are one statement: tcgen05.ld writes its destination registers asynchronously
+// (they hold the data only after tcgen05.wait::ld), while the compiler takes them as the outputs
+// of the statement that issues the load and may read, move or spill them anywhere after it.
+__device__ __forceinline__ void tmem_ld_32x32b_x32_sync(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_ld_wait() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      : "r"(taddr)
+      : "memory");
 }
 
 // ---- paired-CTA (cta_group::2) forms: one warp of each CTA of the pair allocates; the even CTA
