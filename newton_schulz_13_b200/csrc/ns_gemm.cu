@@ -692,13 +692,24 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE>::kThreads, 1)
         }
         return true;
       };
+      // Tensor-memory loads run one chunk ahead: the load of the warp's next active chunk is
+      // issued before the current chunk is processed and waited for after it.
+      auto step = [&](const uint32_t (&cur)[32], uint32_t (&nxt)[32], int i) -> bool {
+        __syncwarp();
+        const bool pre = i + 1 >= i_lo && i + 1 < i_hi;
+        if (pre) tmem_ld_32x32b_x32_issue(tmem_base + tmem_row + tmem_col(ch_of(i + 1)), nxt);
+        const bool ok = chunk(cur, i);
+        if (pre) tmem_ld_wait_regs(nxt);
+        return ok;
+      };
+      uint32_t ra[32], rb[32];
+      __syncwarp();
+      if (i_lo == 0 && i_hi > 0) tmem_ld_32x32b_x32_sync(tmem_base + tmem_row + tmem_col(ch_of(0)), ra);
       bool chunks_ok = true;
 #pragma unroll 1
-      for (int i = 0; i < C::kWarpChunks && chunks_ok; ++i) {
-        uint32_t r[32];
-        __syncwarp();
-        if (i >= i_lo && i < i_hi) tmem_ld_32x32b_x32_sync(tmem_base + tmem_row + tmem_col(ch_of(i)), r);
-        chunks_ok = chunk(r, i);
+      for (int i = 0; i < C::kWarpChunks && chunks_ok; i += 2) {   // kWarpChunks is even
+        chunks_ok = step(ra, rb, i);
+        if (chunks_ok) chunks_ok = step(rb, ra, i + 1);
       }
       if (!chunks_ok) timed_out = true;
       if (timed_out) break;
