@@ -65,7 +65,9 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 //                the two 256-column slots of tensor memory (one accumulator), so the next tile's
 //                MMAs wait for the drain: eight epilogue warps (two per 32-lane quarter of tensor
 //                memory, each taking alternate groups of four 32-column chunks) drain half 0
-//                first, and the next tile's half-0 MMAs overlap the drain of half 1.
+//                first, and the next tile's half-0 MMAs overlap the drain of half 1. At the end
+//                of a tile the last resident K slices also feed half 0 first, so that half 0
+//                completes (tfull[0]) and starts draining while they feed half 1 (tfull[1]).
 template <bool PAIR, bool WIDE = false>
 struct TcCfg {
   static_assert(PAIR || !WIDE, "the wide tile is a CTA-pair tile");
@@ -449,7 +451,10 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE>::kThreads, 1)
             release(stage);
             if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
-          for (uint32_t kb = npre; kb < kblocks; ++kb) {
+          // the last (up to kStages) K slices feed half 0 first, so that half 0 is complete, and
+          // its drain starts, while they still feed half 1
+          const uint32_t npost = kblocks - npre < (uint32_t)C::kStages ? kblocks - npre : (uint32_t)C::kStages;
+          for (uint32_t kb = npre; kb < kblocks - npost; ++kb) {
             if (!mbar_wait_bounded(&full[stage], phase, abort_flag, wait_ns)) {
               timed_out = true;
               break;
@@ -461,7 +466,25 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE>::kThreads, 1)
             if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
           if (timed_out) break;
-          tc_commit_pair_mc(&tfull[0], 0x3);   // the whole tile (both halves)
+          st = stage;
+          ph = phase;
+          for (uint32_t kb = kblocks - npost; kb < kblocks; ++kb) {
+            if (!mbar_wait_bounded(&full[st], ph, abort_flag, wait_ns)) {
+              timed_out = true;
+              break;
+            }
+            tc_fence_after();
+            issue(st, 0, false, kb);
+            if (++st == C::kStages) { st = 0; ph ^= 1u; }
+          }
+          if (timed_out) break;
+          tc_commit_pair_mc(&tfull[0], 0x3);   // half 0 of the tile
+          for (uint32_t kb = kblocks - npost; kb < kblocks; ++kb) {
+            issue(stage, 1, false, kb);
+            release(stage);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          }
+          tc_commit_pair_mc(&tfull[1], 0x3);   // half 1
           acc_phase ^= 1u;
         }
       }
@@ -514,7 +537,7 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE>::kThreads, 1)
       const float alpha = ep.e_acc ? *P.alpha : 1.0f;
       const float s1 = ep.k_acc * alpha_pow(alpha, ep.e_acc);
       const bool has_c = P.tma_c != nullptr && ep.k_c != 0.0f;
-      // the wide tile completes both halves at once, on tfull[0]
+      // the wide tile completes half 0 on tfull[0], half 1 on tfull[1] (waited for in step)
       const bool ok = __all_sync(0xffffffffu,
                                  mbar_wait_bounded(&tfull[WIDE ? 0 : acc], acc_phase, abort_flag, wait_ns));
       if (!ok) {
@@ -696,10 +719,19 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE>::kThreads, 1)
       // issued before the current chunk is processed and waited for after it.
       auto step = [&](const uint32_t (&cur)[32], uint32_t (&nxt)[32], int i) -> bool {
         __syncwarp();
-        const bool pre = i + 1 >= i_lo && i + 1 < i_hi;
+        // wide: the warp's next chunk is the first of half 1, which completes on tfull[1]
+        const bool boundary = WIDE && i == C::kWarpChunks / 2 - 1;
+        const bool pre = !boundary && i + 1 >= i_lo && i + 1 < i_hi;
         if (pre) tmem_ld_32x32b_x32_issue(tmem_base + tmem_row + tmem_col(ch_of(i + 1)), nxt);
-        const bool ok = chunk(cur, i);
+        bool ok = chunk(cur, i);
         if (pre) tmem_ld_wait_regs(nxt);
+        if (boundary && ok) {
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull[1], acc_phase, abort_flag, wait_ns));
+          tc_fence_after();
+          __syncwarp();
+          if (ok && i + 1 >= i_lo && i + 1 < i_hi)
+            tmem_ld_32x32b_x32_sync(tmem_base + tmem_row + tmem_col(ch_of(i + 1)), nxt);
+        }
         return ok;
       };
       uint32_t ra[32], rb[32];
