@@ -987,7 +987,7 @@ int run_ns(DeviceState& ds, Plan& P, const Wave& w, int wave_idx, const std::vec
     }
     if (P.x_bf16) {
       e = timed_launch(MUON_KC_GEMM, s, w.fl_upd, w.ex_upd, [&] {
-        return (w.wide ? launch_gemm_tc_pair_wide : launch_gemm_tc_pair_upd)(tc(upd), n, w.tiles_upd, eu, ds.d_status,
+        return (w.wide ? launch_gemm_tc_pair_wide : launch_gemm_tc_pair)(tc(upd), n, w.tiles_upd, eu, ds.d_status,
                                                                          ds.pair_capacity, s);
       }, MUON_KC_GEMM_UPDATE);
     } else {

@@ -190,9 +190,6 @@ cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_
                            EpiScalars ep, int* status, int grid, cudaStream_t s);
 cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                 EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
-// The same 256 x 256 tiles with eight epilogue warps (the update product of waves of small matrices).
-cudaError_t launch_gemm_tc_pair_upd(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
-                                    EpiScalars ep, int* status, int max_pairs, cudaStream_t s);
 // The same with 256 x kTcWideBN tiles (problem tables built with tiles_n = ceil(N / kTcWideBN)).
 cudaError_t launch_gemm_tc_pair_wide(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                      EpiScalars ep, int* status, int max_pairs, cudaStream_t s);

@@ -9,8 +9,8 @@
 // one launch with tiles claimed in order (see CHAIN below). The Muon step uses the CTA-pair
 // variants (clusters of two CTAs on two SMs, tcgen05 cta_group::2): 256 x 256 tiles, or 256 x 512
 // "wide" tiles for the Gram and update products of large matrices. A single-CTA variant
-// (128 x 256 tiles) serves the no-allocation entry point. 192 threads per CTA (320 for the wide
-// tile, whose epilogue has eight warps):
+// (128 x 256 tiles) serves the no-allocation entry point. 320 threads per CTA for the CTA-pair
+// launches of one phase (eight epilogue warps), 192 for chained launches and the single CTA:
 //   warp 0      TMA producer: 64-deep K slices of opA and opB into a shared-memory ring
 //               (128-byte swizzle), K-major or MN-major boxes per operand; in a pair each CTA
 //               loads its own 128 opA rows and its 128 of every 256 opB rows, and both CTAs'
@@ -19,7 +19,7 @@
 //               accumulation in tensor memory; 256 x 256 tiles alternate between two
 //               accumulators, so the epilogue of one tile overlaps the MMAs of the next, and
 //               wide tiles use both 256-column slots as the two halves of one accumulator;
-//   warps 2-5   epilogue (2-9 for the wide tile): tcgen05.ld of the accumulator, scale, add s_c * C, round to bf16,
+//   warps 2-9   epilogue (2-5 when chained or single-CTA): tcgen05.ld of the accumulator, scale, add s_c * C, round to bf16,
 //               stage 32 x 32 sub-tiles in shared memory and write them with TMA stores (pair),
 //               or store directly (single CTA). For the symmetric products (A = X X^T and
 //               A A = A A^T) only tiles that touch the upper triangle are computed; the output
@@ -68,10 +68,11 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 //                first, and the next tile's half-0 MMAs overlap the drain of half 1. At the end
 //                of a tile the last resident K slices also feed half 0 first, so that half 0
 //                completes (tfull[0]) and starts draining while they feed half 1 (tfull[1]).
-// EPI8 (CTA pair, 256 x 256 tiles): eight epilogue warps, as on the wide tile; used for the update
-// product, whose epilogue is the bottleneck when K is short (K = 768: the MMA thread waited on
-// the accumulators about a quarter of its time with four warps).
-template <bool PAIR, bool WIDE = false, bool EPI8 = false>
+// CTA-pair launches of one phase run eight epilogue warps, two per 32-lane quarter of tensor
+// memory (with four, the 256 x 256 products of short K waited on their epilogue: the MMA thread
+// of the update waited for a free accumulator about a quarter of its time at K = 768). Chained
+// launches keep four (their tile queue has one reader per epilogue warp).
+template <bool PAIR, bool WIDE = false, bool CHAIN = false>
 struct TcCfg {
   static_assert(PAIR || !WIDE, "the wide tile is a CTA-pair tile");
   static constexpr int kTileM = PAIR ? 256 : 128;
@@ -85,7 +86,7 @@ struct TcCfg {
   static constexpr uint32_t kStageBytes = kABytes + kBBytes;
   static constexpr uint32_t kTmemCols = 512;
   // warps: TMA producer, MMA issuer, then the epilogue warps
-  static constexpr int kEpiWarps = (WIDE || EPI8) ? 8 : 4;
+  static constexpr int kEpiWarps = (PAIR && !CHAIN) ? 8 : 4;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kWarpChunks = kTileN / 32 / (kEpiWarps / 4);   // 32-column chunks per warp and tile
   static_assert(kWarpChunks * 32 * (kEpiWarps / 4) == kTileN, "chunks per warp");
@@ -93,7 +94,7 @@ struct TcCfg {
   static constexpr uint32_t kEpiArrivals = PAIR ? 2 * kEpiWarps : kEpiWarps;
   // CTA pair: staging per epilogue warp in 2 KB slots (a 32 x 32 bf16 sub-tile each; two make a
   // slot for an fp32 sub-tile or a sub-tile and its mirror), 32 KB in all
-  static constexpr uint32_t kSlots = (WIDE || EPI8) ? 2 : 4;
+  static constexpr uint32_t kSlots = kEpiWarps == 8 ? 2 : 4;
   static constexpr uint32_t kStagingPerWarp = kSlots * 2048;
   static constexpr uint32_t kStagingBytes = PAIR ? kEpiWarps * kStagingPerWarp : 0;
   static constexpr size_t kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 512;
@@ -131,13 +132,12 @@ constexpr uint32_t kNoTile = 0xffffffffu;
 // matrix) before its operands are loaded, and each epilogue warp counts its finished tiles. A
 // claimed tile depends only on tiles claimed before it, so the launch makes progress whether or
 // not all of its CTAs are resident.
-template <bool PAIR, bool WIDE, bool CHAIN, bool EPI8 = false>
-__global__ void __launch_bounds__(TcCfg<PAIR, WIDE, EPI8>::kThreads, 1)
+template <bool PAIR, bool WIDE, bool CHAIN>
+__global__ void __launch_bounds__(TcCfg<PAIR, WIDE, CHAIN>::kThreads, 1)
     ns_gemm_tc_kernel(const GemmProblem* __restrict__ probs, int nprobs, uint32_t total_tiles,
                       EpiScalars ep, int* __restrict__ status, ChainArgs ca) {
   static_assert(!CHAIN || (PAIR && !WIDE), "chained launches use 256 x 256 CTA-pair tiles");
-  static_assert(!EPI8 || (PAIR && !WIDE && !CHAIN), "eight-warp 256 x 256 epilogue: per-phase pair launches");
-  using C = TcCfg<PAIR, WIDE, EPI8>;
+  using C = TcCfg<PAIR, WIDE, CHAIN>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE, EPI8>::kThreads, 1)
     const uint32_t quarter = (uint32_t)(warp & 3);
     const uint32_t sub = (uint32_t)(warp - 2) >> 2;   // wide tile: which groups of four chunks
     auto ch_of = [&](int i) -> int {
-      return WIDE ? ((i >> 2) << 3) + (int)(sub << 2) + (i & 3) : (EPI8 ? (int)(sub << 2) + i : i);
+      return WIDE ? ((i >> 2) << 3) + (int)(sub << 2) + (i & 3) : (C::kEpiWarps == 8 ? (int)(sub << 2) + i : i);
     };
     uint8_t* stg = staging + (uint32_t)(warp - 2) * C::kStagingPerWarp;
     uint64_t* cbar = drain + 1 + C::kSlots * (warp - 2);   // this warp's operand-load barriers, one per slot
@@ -915,12 +915,12 @@ cudaError_t launch_gemm_tc(const GemmProblem* probs, int nprobs, uint32_t total_
 
 namespace {
 
-template <bool WIDE, bool CHAIN, bool EPI8 = false>
+template <bool WIDE, bool CHAIN>
 cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles, EpiScalars ep,
                         int* status, int max_pairs, cudaStream_t s, ChainArgs ca) {
-  using C = TcCfg<true, WIDE, EPI8>;
+  using C = TcCfg<true, WIDE, CHAIN>;
   static PerDeviceOnce once;   // one per instantiation
-  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<true, WIDE, CHAIN, EPI8>, (int)C::kSmemBytes, once);
+  cudaError_t e = set_smem_limit((const void*)ns_gemm_tc_kernel<true, WIDE, CHAIN>, (int)C::kSmemBytes, once);
   if (e != cudaSuccess) return e;
   if (total_tiles == 0) return cudaSuccess;
   const uint32_t pairs = (uint32_t)max_pairs < total_tiles ? (uint32_t)max_pairs : total_tiles;
@@ -936,8 +936,7 @@ cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_til
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, ns_gemm_tc_kernel<true, WIDE, CHAIN, EPI8>, probs, nprobs, total_tiles, ep, status,
-                            ca);
+  return cudaLaunchKernelEx(&cfg, ns_gemm_tc_kernel<true, WIDE, CHAIN>, probs, nprobs, total_tiles, ep, status, ca);
 }
 
 }  // namespace
@@ -945,11 +944,6 @@ cudaError_t launch_pair(const GemmProblem* probs, int nprobs, uint32_t total_til
 cudaError_t launch_gemm_tc_pair(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
                                 EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
   return launch_pair<false, false>(probs, nprobs, total_tiles, ep, status, max_pairs, s, ChainArgs{});
-}
-
-cudaError_t launch_gemm_tc_pair_upd(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
-                                    EpiScalars ep, int* status, int max_pairs, cudaStream_t s) {
-  return launch_pair<false, false, true>(probs, nprobs, total_tiles, ep, status, max_pairs, s, ChainArgs{});
 }
 
 cudaError_t launch_gemm_tc_pair_wide(const GemmProblem* probs, int nprobs, uint32_t total_tiles,
