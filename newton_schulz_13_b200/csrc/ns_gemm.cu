@@ -500,7 +500,7 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE, CHAIN>::kThreads, 1)
     }
     __syncwarp();
   } else if constexpr (PAIR) {
-    // ------------------------------------------------------------ epilogue warps 2..5 (pair)
+    // ------------------------------------------------------------ epilogue warps 2..9 (pair; 2..5 chained)
     // Each warp owns 32 accumulator rows. Per 32-column chunk it forms
     //   D = k_acc alpha^e acc + k_c C + diag I
     // in fp32, rounds to bf16, stages the 32 x 32 sub-tile in shared memory (64-byte swizzle) and
