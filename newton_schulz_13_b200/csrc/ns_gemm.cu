@@ -501,7 +501,8 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE, CHAIN>::kThreads, 1)
     __syncwarp();
   } else if constexpr (PAIR) {
     // ------------------------------------------------------------ epilogue warps 2..9 (pair; 2..5 chained)
-    // Each warp owns 32 accumulator rows. Per 32-column chunk it forms
+    // Each warp owns 32 accumulator rows (a 32-lane quarter of tensor memory; with eight warps,
+    // two share a quarter and split its columns). Per 32-column chunk it forms
     //   D = k_acc alpha^e acc + k_c C + diag I
     // in fp32, rounds to bf16, stages the 32 x 32 sub-tile in shared memory (64-byte swizzle) and
     // writes it with a TMA store; rows and columns past the matrix are clipped by the store. A
@@ -509,10 +510,11 @@ __global__ void __launch_bounds__(TcCfg<PAIR, WIDE, CHAIN>::kThreads, 1)
     // staged transposed and stored at the mirrored position, those strictly below are skipped)
     // or in the upper-block form (sym 2: chunks in a 256-block below the diagonal are skipped).
     // The chunks a tile writes ("active") are one contiguous range.
-    // A warp takes 8 of the tile's 32-column chunks: all of them (256-column tile), or (wide
-    // tile, two warps per quarter) alternate groups of four, so that half 0 is drained first by
-    // both. The warp's active chunks are one contiguous run of its own list.
-    // Staging is a ring of 2 KB slots per warp (four; two for the wide tile's eight warps) that the
+    // A warp's chunks: all eight of a 256-column tile (four warps, chained); with two warps per
+    // quarter, chunks 0-3 or 4-7 of a 256-column tile, or alternate groups of four of a 512-column
+    // tile, so that half 0 is drained first by both. The warp's active chunks are one contiguous
+    // run of its own list.
+    // Staging is a ring of 2 KB slots per warp (four with four warps, two with eight) that the
     // active chunks use in turn: one slot per bf16 sub-tile, or pairs of slots for the fused last
     // update (fp32 parameter sub-tiles) and for whole symmetric outputs (a sub-tile and its
     // mirror). A chunk that reads an operand sub-tile (the addend C, or the parameters) has its
