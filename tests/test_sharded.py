@@ -56,6 +56,41 @@ def test_layout_places_every_matrix_in_its_group_and_owner_slot():
         sharded.ShardedLayout(shapes, 2, group_elements=0)
 
 
+def test_layout_invariants_on_random_shape_lists():
+    """Any list of shapes, rank count and group size: every matrix sits inside its owner's slot
+    of its group, no two views overlap, each matrix is in exactly one group of its owner, and the
+    views have the matrices' shapes."""
+    import random
+    rng = random.Random(1234)
+    for trial in range(60):
+        n = rng.randint(1, 40)
+        shapes = [(rng.randint(1, 3000), rng.randint(1, 3000)) for _ in range(n)]
+        world = rng.randint(1, 8)
+        total = sum(r * c for r, c in shapes)
+        group = rng.choice([1 << 28, max(1, total // rng.randint(1, 12)), rng.randint(1, 5000)])
+        L = sharded.ShardedLayout(shapes, world, group_elements=group)
+        seen = {}
+        for rk in range(world):
+            assert len(L.groups[rk]) == L.n_groups
+            for g, mats in enumerate(L.groups[rk]):
+                for j in mats:
+                    assert j not in seen, (trial, j)
+                    seen[j] = (rk, g)
+        assert sorted(seen) == list(range(n))
+        spans = []
+        for j, (r, c) in enumerate(shapes):
+            rk, g = seen[j]
+            assert rk == L.owner[j] and g == L.group_of[j]
+            slot0 = L.block_off[g] + rk * L.cap[g]
+            assert slot0 <= L.offset[j] and L.offset[j] + r * c <= slot0 + L.cap[g], (trial, j)
+            spans.append((L.offset[j], L.offset[j] + r * c))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:])), trial
+        assert L.total == sum(world * cap for cap in L.cap)
+        views = L.views(torch.zeros(L.total))
+        assert [tuple(v.shape) for v in views] == shapes
+
+
 def test_expected_exchange_time():
     shapes = synth.WORKLOADS["llama8b"].shapes
     # 28 GB of fp32 parameters; at 8 ranks each receives 7/8 of them
