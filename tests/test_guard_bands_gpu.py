@@ -106,3 +106,36 @@ def test_orthogonalize_writes_stay_inside_the_output(shape, prec, tol, out):
     got = host64(X.view)
     # a bf16 output adds one rounding (2^-9 relative) to the bf16 or fp32 working precision
     assert rel(got, want) <= (tol if out == "fp32" else tol + 4e-3), rel(got, want)
+
+
+@pytest.mark.parametrize("prec,tol", [("bf16", TOL_O_BF16), ("fp32", TOL_O_FP32)], ids=["bf16", "fp32"])
+def test_mixed_wave_on_wide_tiles(prec, tol):
+    """One call whose wave runs on 256 x 512 tiles (the 2100 x 2600 matrix carries its FLOPs) and
+    also holds matrices whose contraction is a single K slice or a few (1 x 7, 7 x 1, 33 x 17,
+    300 x 64): their tiles start and end inside the ring's first stages. Each matrix in its own
+    guard bands, values against the oracle."""
+    import newton_schulz_13_b200 as ns
+    shapes = [(7, 1), (2100, 2600), (33, 17), (1, 7), (300, 64)]
+    rng = np.random.default_rng(71)
+    p0s, gs, Ps, Ms, Gs = [], [], [], [], []
+    for k, (r, c) in enumerate(shapes):
+        p0 = synth.round_to(0.02 * rng.standard_normal((r, c)), "fp32")
+        g = synth.round_to(rng.standard_normal((r, c)), "bf16")
+        p0s.append(p0)
+        gs.append(g)
+        Ps.append(Banded(p0, torch.float32, k % 3))
+        Ms.append(Banded(np.zeros((r, c)), torch.float32, 1))
+        Gs.append(Banded(g, torch.bfloat16, 2))
+    ns.muon_step([P.view for P in Ps], [G.view for G in Gs], [M.view for M in Ms], lr=0.02, mu=0.95,
+                 nesterov=True, weight_decay=0.1, rms_scale=1, steps=5, coeffs=Q5, eps=1e-7, prec=prec)
+    torch.cuda.synchronize()
+    assert ns.check_status() == ns.OK
+    for k, (r, c) in enumerate(shapes):
+        assert Ps[k].bands_intact() and Ms[k].bands_intact() and Gs[k].unchanged(), shapes[k]
+        o_p, o_m = p0s[k].astype(np.float64).copy(), np.zeros((r, c))
+        O_ref = ns_blas.muon_step([o_p], [gs[k]], [o_m], lr=0.02, mu=0.95, nesterov=True, weight_decay=0.1,
+                                  rms_mode=1, coeffs=Q5, zero_center=False, eps=1e-7, want_O=True)[0]
+        s = np.sqrt(max(1.0, r / c))
+        decay = np.float64(np.float32(1.0 - np.float32(0.02) * np.float32(0.1)))
+        O_gpu = (p0s[k] * decay - host64(Ps[k].view)) / (np.float64(np.float32(0.02)) * s)
+        assert rel(O_gpu, O_ref) <= tol, (shapes[k], rel(O_gpu, O_ref))
