@@ -45,13 +45,26 @@ def _step(ns, p0, g, prec):
     return p
 
 
-# 256 x 512: the 256 x 256 CTA-pair tiles; 2100 x 2600: the 256 x 512 tiles; fp32: the 3xTF32 kernel
-@pytest.mark.parametrize("shape,prec,tol", [((256, 512), "bf16", TOL_O_BF16), ((2100, 2600), "bf16", TOL_O_BF16),
-                                            ((256, 512), "fp32", TOL_O_FP32), ((700, 300), "fp32", TOL_O_FP32)],
-                         ids=["bf16-256x512", "bf16-wide-2100x2600", "fp32-256x512", "fp32-tall-700x300"])
-def test_wait_that_runs_out_is_reported_and_the_device_recovers(short_waits, shape, prec, tol):
+# 256 x 512: the 256 x 256 CTA-pair tiles, in one chained launch (chain 1, the default for a single
+# small matrix) or in one launch per phase with eight epilogue warps (chain 0); 2100 x 2600: the
+# 256 x 512 tiles; fp32: the 3xTF32 kernel
+@pytest.mark.parametrize("shape,prec,tol,chain", [((256, 512), "bf16", TOL_O_BF16, 1), ((256, 512), "bf16", TOL_O_BF16, 0),
+                                                  ((2100, 2600), "bf16", TOL_O_BF16, 1),
+                                                  ((256, 512), "fp32", TOL_O_FP32, 1), ((700, 300), "fp32", TOL_O_FP32, 1)],
+                         ids=["bf16-256x512-chained", "bf16-256x512-per-phase", "bf16-wide-2100x2600", "fp32-256x512",
+                              "fp32-tall-700x300"])
+def test_wait_that_runs_out_is_reported_and_the_device_recovers(short_waits, shape, prec, tol, chain):
     import newton_schulz_13_b200 as ns
+    ns.set_chained_launch(chain)
+    try:
+        _timeout_then_recover(ns, shape, prec, tol)
+    finally:
+        ns.set_chained_launch(1)
+
+
+def _timeout_then_recover(ns, shape, prec, tol):
     p0, g = _inputs(shape, 71)
+    short_waits = ns.set_wait_limit_ns
     short_waits(4)                                    # 4 ns: the first incomplete wait gives up
     _step(ns, p0, g, prec)
     with pytest.raises(ns.MuonError) as ei:
